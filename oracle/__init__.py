@@ -1,0 +1,8 @@
+"""fp64 CPU oracle of the CSA / HCA attention layer (test infrastructure only).
+
+Only `tests/`, `__graft_entry__.smoke()` and `bench.py`'s CPU-baseline legs
+may import this package.  It shares no code with the CUDA path.
+"""
+from .csa_oracle import (  # noqa: F401
+    attend, compress, csa_prefill_layer, gather_rows, hca_attn, index_scores, index_topk,
+    n_compressed, n_visible, rope, rotate_raw, sparse_attn, topk_select, window_tokens)

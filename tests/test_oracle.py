@@ -1,0 +1,325 @@
+"""Pins of the fp64 oracle against what the pages and mathematics fix.
+
+None of these tests retypes the oracle's formulas: they use closed forms,
+invariants, a library routine the method reduces to (torch SDPA in float64),
+an independent pure-Python brute force (tests/brute.py) and the entry counts
+the workloads state (tests/golden/entry_counts.txt).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import brute
+import oracle
+from oracle import csa_oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+THETA = 10000.0
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- counts
+def test_entry_counts_match_stated_workloads():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "entry_counts.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert len(rows) == 5
+    for T, w, s, n in (map(int, r) for r in rows):
+        assert oracle.n_compressed(T, w, s) == n
+
+
+def test_visibility_counts():
+    # decode query at the last context token sees every pooled entry
+    assert oracle.n_visible(65535, 16383, 8, 4) == 16383
+    assert oracle.n_visible(1048575, 262143, 8, 4) == 262143
+    assert oracle.n_visible(131071, 1024, 128, 128) == 1024
+    # an entry is visible once its last (8th) token has been seen
+    assert oracle.n_visible(6, 100, 8, 4) == 0
+    assert oracle.n_visible(7, 100, 8, 4) == 1
+    assert oracle.n_visible(10, 100, 8, 4) == 1
+    assert oracle.n_visible(11, 100, 8, 4) == 2
+    for t in range(0, 80):
+        assert oracle.n_visible(t, 1000, 8, 4) == len(brute.visible(t, 1000, 8, 4))
+
+
+def test_window_tokens():
+    assert list(oracle.window_tokens(5, 16, 0, 256)) == list(range(0, 6))
+    assert list(oracle.window_tokens(300, 16, 0, 1000)) == list(range(285, 301))
+    assert list(oracle.window_tokens(65535, 128, 65408, 128)) == list(range(65408, 65536))
+    for t in (0, 3, 17, 40):
+        assert list(oracle.window_tokens(t, 16, 10, 20)) == brute.window(t, 16, 10, 20)
+
+
+# ---------------------------------------------------------------- RoPE
+def test_rope_is_complex_rotation():
+    x = _rng(0).standard_normal((5, 32))
+    pos = np.array([0, 1, 7, 1000, 65535])
+    r = 16
+    got = oracle.rope(x, pos, r, THETA)
+    assert np.array_equal(got[:, :16], x[:, :16])  # leading dims untouched
+    i = np.arange(r // 2)
+    z = (x[:, 16::2] + 1j * x[:, 17::2]) * np.exp(1j * np.outer(pos, THETA ** (-2.0 * i / r)))
+    np.testing.assert_allclose(got[:, 16::2], z.real, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[:, 17::2], z.imag, rtol=0, atol=1e-12)
+
+
+def test_rope_relative_distance_and_inverse():
+    rng = _rng(1)
+    a, b = rng.standard_normal(64), rng.standard_normal(64)
+    dots = [oracle.rope(a, p, 64, THETA) @ oracle.rope(b, p - 37, 64, THETA)
+            for p in (40, 1000, 123456)]
+    np.testing.assert_allclose(dots, dots[0], rtol=0, atol=1e-9)
+    back = oracle.rope(oracle.rope(a, 777, 64, THETA), -777, 64, THETA)
+    np.testing.assert_allclose(back, a, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- compress
+def test_uniform_gates_make_exact_mean_pooling():
+    rng = _rng(2)
+    x = rng.standard_normal((40, 24))
+    g = np.full((40, 24), 0.37)
+    e = oracle.compress(x, g, 8, 4, 0, THETA)
+    assert e.shape == (9, 24)
+    for j in range(9):
+        np.testing.assert_allclose(e[j], x[4 * j:4 * j + 8].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_dominant_gate_copies_one_tap():
+    rng = _rng(3)
+    x = rng.standard_normal((24, 16))
+    g = np.zeros((24, 16))
+    g[np.arange(24) % 4 == 1] = 800.0  # tap u=1 of every entry dominates
+    e = oracle.compress(x, g, 8, 4, 0, THETA)
+    # taps 1 and 5 of each window both carry the large logit: equal halves
+    for j in range(e.shape[0]):
+        np.testing.assert_allclose(e[j], 0.5 * (x[4 * j + 1] + x[4 * j + 5]), atol=1e-12)
+
+
+def test_compress_matches_brute_force():
+    rng = _rng(4)
+    for (T, d, w, s, r) in ((19, 16, 8, 4, 8), (20, 8, 4, 4, 4), (9, 6, 2, 2, 2)):
+        x, g = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+        got = oracle.compress(x, g, w, s, r, THETA, pos_offset=3)
+        ref = np.array(brute.compress(x.tolist(), g.tolist(), w, s, r, THETA, 3))
+        assert got.shape == ref.shape
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- indexer
+def test_index_scores_integer_exact_and_brute():
+    rng = _rng(5)
+    q = rng.integers(-8, 9, size=(3, 4, 16)).astype(np.float64)
+    k = rng.integers(-8, 9, size=(21, 16)).astype(np.float64)
+    w = np.exp2(rng.integers(-2, 3, size=(3, 4))).astype(np.float64)
+    got = oracle.index_scores(q, w, k)
+    for t in range(3):
+        ref = brute.scores(q[t].tolist(), w[t].tolist(), k.tolist())
+        assert got[t].tolist() == ref  # integers times powers of two: exact
+        # exact integer arithmetic, times 4 to clear the 2^-2 weights
+        exact = [sum(int(w[t, h] * 4) * max(0, int(q[t, h] @ k[j])) for h in range(4))
+                 for j in range(21)]
+        assert (got[t] * 4).astype(np.int64).tolist() == exact
+
+
+def test_topk_ties_and_order():
+    rng = _rng(6)
+    for trial in range(30):
+        n = int(rng.integers(1, 60))
+        s = rng.integers(0, 5, size=n).astype(np.float64)  # many ties
+        k = int(rng.integers(1, 20))
+        nv = int(rng.integers(0, n + 1))
+        got = oracle.topk_select(s, nv, k)
+        assert got.tolist() == brute.topk(s.tolist(), nv, k)
+
+
+def test_topk_fewer_visible_keeps_all_and_pads():
+    s = np.array([5.0, 1.0, 9.0, 2.0])
+    assert oracle.topk_select(s, 3, 8).tolist() == [0, 1, 2, -1, -1, -1, -1, -1]
+    assert oracle.topk_select(s, 0, 2).tolist() == [-1, -1]
+    # negative zero ties with positive zero, lower index wins
+    z = np.array([0.0, -0.0, 0.0, -0.0])
+    assert oracle.topk_select(z, 4, 2).tolist() == [0, 1]
+
+
+# ---------------------------------------------------------------- attention
+def test_attention_reduces_to_sdpa():
+    """sink -> -inf, no RoPE, every entry selected: plain softmax attention."""
+    rng = _rng(7)
+    H, d, R = 3, 32, 11
+    q = rng.standard_normal((H, d))
+    rows = rng.standard_normal((R, d))
+    scale = 1 / math.sqrt(d)
+    got = oracle.attend(q, 5, rows, np.full(H, -np.inf), scale, 0, THETA)
+    tq = torch.from_numpy(q)[None, :, None, :]           # [1, H, 1, d]
+    tk = torch.from_numpy(rows)[None, None].expand(1, H, R, d)
+    mask = torch.ones(1, H, 1, R, dtype=torch.bool)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tk, attn_mask=mask,
+                                                           scale=scale)
+    np.testing.assert_allclose(got, ref[0, :, 0].numpy(), rtol=0, atol=1e-12)
+
+
+def test_single_key_closed_form():
+    """One visible entry, no window, sink -> -inf: o = R(p_j - t) e_j."""
+    rng = _rng(8)
+    d, r = 32, 16
+    e = rng.standard_normal(d)
+    pj, t = 12, 40
+    row = oracle.rope(e[None], pj, r, THETA)
+    q = rng.standard_normal((2, d))
+    got = oracle.attend(q, t, row, np.full(2, -np.inf), 0.1, r, THETA)
+    i = np.arange(r // 2)
+    zz = (e[16::2] + 1j * e[17::2]) * np.exp(1j * (pj - t) * THETA ** (-2.0 * i / r))
+    for h in range(2):
+        np.testing.assert_allclose(got[h, :16], e[:16], atol=1e-12)
+        np.testing.assert_allclose(got[h, 16::2], zz.real, atol=1e-12)
+        np.testing.assert_allclose(got[h, 17::2], zz.imag, atol=1e-12)
+
+
+def test_sink_closed_form_and_weight_sum():
+    """q = 0 makes every logit 0: each of n rows weighs 1/(e^sink + n)."""
+    d, n = 16, 7
+    rows = np.zeros((n, d))
+    rows[:, :8] = 1.0  # value 1 in the un-rotated dims, 0 in the rope dims
+    sink = np.array([-np.inf, 0.0, 1.5, -2.0])
+    got = oracle.attend(np.zeros((4, d)), 9, rows, sink, 0.25, 8, THETA)
+    for h in range(4):
+        want = n / (math.exp(sink[h]) + n) if np.isfinite(sink[h]) else 1.0
+        np.testing.assert_allclose(got[h, :8], want, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(got[h, 8:], 0.0, atol=1e-14)
+    assert got[0, 0] == pytest.approx(1.0, abs=1e-15)  # weights sum to 1
+    assert np.all(got[1:, 0] < 1.0)                     # finite sink: below 1
+    # random logits: the weight sum (value rows of ones) stays below 1
+    rng = _rng(9)
+    got2 = oracle.attend(rng.standard_normal((4, d)), 9, rows, sink, 0.25, 8, THETA)
+    assert got2[0, 0] == pytest.approx(1.0, abs=1e-14)
+    assert np.all(got2[1:, 0] < 1.0)
+
+
+def test_attention_matches_brute_force():
+    rng = _rng(10)
+    H, d, r = 2, 12, 4
+    q = rng.standard_normal((H, d))
+    rows = rng.standard_normal((6, d))
+    sink = rng.standard_normal(H)
+    got = oracle.attend(q, 17, rows, sink, 0.3, r, THETA)
+    ref = brute.attend(q.tolist(), 17, rows.tolist(), sink.tolist(), 0.3, r, THETA)
+    np.testing.assert_allclose(got, np.array(ref), rtol=0, atol=1e-12)
+
+
+def _tiny_layer(seed, T=64, d=16, r=8, H=2, HI=2, dI=8, k=5, W=6, width=8, stride=4):
+    rng = _rng(seed)
+    return dict(
+        x=rng.standard_normal((T, d)), g=rng.standard_normal((T, d)),
+        q_idx=rng.integers(-3, 4, size=(T, HI, dI)).astype(np.float64),
+        w=np.exp2(rng.integers(-1, 2, size=(T, HI))).astype(np.float64),
+        k_idx=rng.integers(-3, 4, size=((T - width) // stride + 1, dI)).astype(np.float64),
+        q=rng.standard_normal((T, H, d)), sink=rng.standard_normal(H),
+        kw=dict(width=width, stride=stride, topk=k, window=W, rope_dim=r, theta=THETA,
+                scale=1 / math.sqrt(d)))
+
+
+def test_whole_layer_matches_brute_force():
+    L = _tiny_layer(11)
+    kw = L["kw"]
+    kv_cmp, kv_raw, idx, out = oracle.csa_prefill_layer(
+        L["x"], L["g"], L["q_idx"], L["w"], L["k_idx"], L["q"], L["sink"], **kw)
+    b_cmp = brute.compress(L["x"].tolist(), L["g"].tolist(), kw["width"], kw["stride"],
+                           kw["rope_dim"], THETA)
+    np.testing.assert_allclose(kv_cmp, np.array(b_cmp), atol=1e-12)
+    T = L["x"].shape[0]
+    for t in range(T):
+        sc = brute.scores(L["q_idx"][t].tolist(), L["w"][t].tolist(), L["k_idx"].tolist())
+        vis = brute.visible(t, len(b_cmp), kw["width"], kw["stride"])
+        sel = brute.topk(sc, len(vis), kw["topk"])
+        assert idx[t].tolist() == sel
+        raw = [brute._rot(list(L["x"][u]), u, kw["rope_dim"], THETA)
+               for u in brute.window(t, kw["window"], 0, T)]
+        rows = [b_cmp[j] for j in sel if j >= 0] + raw
+        ref = brute.attend(L["q"][t].tolist(), t, rows, L["sink"].tolist(), kw["scale"],
+                           kw["rope_dim"], THETA)
+        np.testing.assert_allclose(out[t], np.array(ref), atol=1e-12)
+
+
+def test_sparse_equals_dense_when_k_covers_all():
+    L = _tiny_layer(12, k=100)
+    kw = L["kw"]
+    kv_cmp, kv_raw, idx, out = oracle.csa_prefill_layer(
+        L["x"], L["g"], L["q_idx"], L["w"], L["k_idx"], L["q"], L["sink"], **kw)
+    T = L["x"].shape[0]
+    dense = oracle.hca_attn(L["q"], np.arange(T), kv_cmp, kv_cmp.shape[0], kv_raw, 0, T,
+                            L["sink"], kw["scale"], kw["window"], kw["width"], kw["stride"],
+                            kw["rope_dim"], THETA)
+    np.testing.assert_allclose(out, dense, rtol=0, atol=1e-13)
+
+
+def test_hca_is_csa_path_with_128_pooling():
+    rng = _rng(13)
+    T, d, H = 600, 16, 2
+    x, g = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    q, sink = rng.standard_normal((T, H, d)), rng.standard_normal(H)
+    kv = oracle.compress(x, g, 128, 128, 8, THETA)
+    raw = oracle.rotate_raw(x, 0, 8, THETA)
+    rows = np.array([0, 126, 127, 128, 300, 599])
+    a = oracle.hca_attn(q, np.arange(T), kv, kv.shape[0], raw, 0, T, sink, 0.25, 128,
+                        128, 128, 8, THETA, rows)
+    all_idx = np.tile(np.arange(64), (T, 1))
+    all_idx = np.where(all_idx < np.array([oracle.n_visible(t, kv.shape[0], 128, 128)
+                                           for t in range(T)])[:, None], all_idx, -1)
+    b = oracle.sparse_attn(q, np.arange(T), kv, all_idx, raw, 0, T, sink, 0.25, 128, 8,
+                           THETA, rows)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-14)
+
+
+def test_shift_of_all_positions_leaves_output_unchanged():
+    L = _tiny_layer(14)
+    kw = L["kw"]
+    T = L["x"].shape[0]
+    outs = []
+    for shift in (0, 1000, 77777):
+        kv_cmp = oracle.compress(L["x"], L["g"], kw["width"], kw["stride"], kw["rope_dim"],
+                                 THETA, pos_offset=shift)
+        kv_raw = oracle.rotate_raw(L["x"], shift, kw["rope_dim"], THETA)
+        idx = oracle.index_topk(L["q_idx"], L["w"], L["k_idx"], np.arange(T), kv_cmp.shape[0],
+                                kw["width"], kw["stride"], kw["topk"])
+        res = []
+        for t in range(T):
+            rows = oracle.gather_rows(kv_cmp, idx[t], kv_raw, t, kw["window"], 0, T)
+            res.append(oracle.attend(L["q"][t], t + shift, rows, L["sink"], kw["scale"],
+                                     kw["rope_dim"], THETA))
+        outs.append(np.stack(res))
+    np.testing.assert_allclose(outs[1], outs[0], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(outs[2], outs[0], rtol=0, atol=1e-9)
+
+
+# ---------------------------------------------------------------- planted mistakes
+def test_pins_catch_planted_mistakes(monkeypatch):
+    """A wrong rotation sign or a dropped sink term in the oracle must trip a pin."""
+    good_rope = csa_oracle.rope
+
+    def bad_rope(x, pos, rope_dim, theta):
+        return good_rope(x, -np.asarray(pos), rope_dim, theta)
+
+    monkeypatch.setattr(csa_oracle, "rope", bad_rope)
+    monkeypatch.setattr(oracle, "rope", bad_rope)
+    with pytest.raises(AssertionError):
+        test_rope_is_complex_rotation()
+    with pytest.raises(AssertionError):
+        test_single_key_closed_form()
+    monkeypatch.setattr(csa_oracle, "rope", good_rope)
+    monkeypatch.setattr(oracle, "rope", good_rope)
+
+    good_attend = csa_oracle.attend
+
+    def no_sink(q, t, rows, sink, scale, rope_dim, theta):
+        return good_attend(q, t, rows, np.full_like(np.asarray(sink, float), -np.inf), scale,
+                           rope_dim, theta)
+
+    monkeypatch.setattr(csa_oracle, "attend", no_sink)
+    monkeypatch.setattr(oracle, "attend", no_sink)
+    with pytest.raises(AssertionError):
+        test_sink_closed_form_and_weight_sum()
