@@ -150,8 +150,8 @@ def index_scores(q_idx: np.ndarray, w: np.ndarray, k_idx: np.ndarray) -> np.ndar
     q_idx = np.asarray(q_idx, dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
     k_idx = np.asarray(k_idx, dtype=np.float64)
-    dots = np.einsum("thc,jc->thj", q_idx, k_idx)
-    return np.einsum("th,thj->tj", w, np.maximum(dots, 0.0))
+    dots = np.matmul(q_idx, k_idx.T)                      # [Tq, H_I, N]
+    return np.matmul(w[:, None, :], np.maximum(dots, 0.0))[:, 0, :]
 
 
 def topk_select(scores: np.ndarray, n_vis: int, k: int) -> np.ndarray:
@@ -217,8 +217,8 @@ def gather_rows(kv_cmp_b: np.ndarray, sel: np.ndarray, kv_raw_b: np.ndarray, t: 
     sel = np.asarray(sel, dtype=np.int64)
     sel = sel[sel >= 0]
     win = window_tokens(t, window, raw_pos0, n_raw)
-    parts = [np.asarray(kv_cmp_b, dtype=np.float64)[sel],
-             np.asarray(kv_raw_b, dtype=np.float64)[win - raw_pos0]]
+    parts = [np.asarray(kv_cmp_b)[sel].astype(np.float64),
+             np.asarray(kv_raw_b)[win - raw_pos0].astype(np.float64)]
     return np.concatenate(parts, axis=0)
 
 

@@ -1,0 +1,248 @@
+"""ctypes binding of libcsa.so (the C ABI in include/csa.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  Functions take torch CUDA tensors (torch is used for device
+memory and streams), check dtype / contiguity / device, and pass raw
+pointers and sizes through.  A missing library raises immediately: there is
+no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_F32, CSA_BF16 = 0, 1
+CSA_OP_COMPRESS, CSA_OP_INDEX_TOPK, CSA_OP_SPARSE_ATTN, CSA_OP_HCA_ATTN, CSA_OP_TOPK_SELECT = range(5)
+
+STATUS = {
+    0: "CSA_OK", 1: "CSA_ERR_INVALID_ARGUMENT", 2: "CSA_ERR_MISALIGNED",
+    3: "CSA_ERR_UNSUPPORTED_SHAPE", 4: "CSA_ERR_UNSUPPORTED_DEVICE",
+    5: "CSA_ERR_WORKSPACE_TOO_SMALL", 6: "CSA_ERR_CUDA", 7: "CSA_ERR_DEVICE_TIMEOUT",
+    8: "CSA_ERR_DEVICE_BOUNDS",
+}
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+class csa_params_t(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("rope_dim", ctypes.c_int32), ("theta", ctypes.c_float),
+                ("scale", ctypes.c_float), ("n_heads", ctypes.c_int32),
+                ("idx_heads", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("window", ctypes.c_int32), ("width", ctypes.c_int32),
+                ("stride", ctypes.c_int32), ("pos_offset", ctypes.c_int32)]
+
+
+@dataclass(frozen=True)
+class Params:
+    """Layer constants (defaults: the measured model's CSA layer)."""
+    d: int = 512
+    rope_dim: int = 64
+    theta: float = 10000.0
+    scale: float | None = None  # None -> 1/sqrt(d)
+    n_heads: int = 128
+    idx_heads: int = 64
+    idx_dim: int = 128
+    topk: int = 1024
+    window: int = 128
+    width: int = 8
+    stride: int = 4
+    pos_offset: int = 0
+
+    def c(self) -> csa_params_t:
+        sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+        return csa_params_t(self.d, self.rope_dim, self.theta, sc, self.n_heads, self.idx_heads,
+                            self.idx_dim, self.topk, self.window, self.width, self.stride,
+                            self.pos_offset)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_PP = ctypes.POINTER(csa_params_t)
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"CUDA library {LIB_PATH} is not built; run "
+                          "sparse_compressed_attention_csa_b200.build.build() (there is no "
+                          "CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.csa_abi_version.restype = ctypes.c_int
+    lib.csa_status_string.restype = ctypes.c_char_p
+    lib.csa_status_string.argtypes = [ctypes.c_int]
+    lib.csa_last_error_detail.restype = ctypes.c_char_p
+    lib.csa_workspace_size.argtypes = [_PP, ctypes.c_int, _I, _I, _I,
+                                       ctypes.POINTER(ctypes.c_size_t)]
+    lib.csa_compress.argtypes = [_PP, ctypes.c_int, _P, _P, _I, _I, _P, _P, _P]
+    lib.csa_index_scores.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]
+    lib.csa_topk_select.argtypes = [_PP, _P, _P, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]
+    lib.csa_index_topk.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P,
+                                   ctypes.c_size_t, _P]
+    lib.csa_sparse_attn.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P,
+                                    _I, _I, _P, _P, ctypes.c_size_t, _P]
+    lib.hca_attn.argtypes = list(lib.csa_sparse_attn.argtypes)
+    lib.csa_poll_device_error.argtypes = [_P]
+    for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
+              "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error"):
+        getattr(lib, f).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def lib():
+    return _load()
+
+
+def _check(st: int):
+    if st != 0:
+        raise CsaError(st, _load().csa_last_error_detail().decode(errors="replace"))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return CSA_BF16
+    if t.dtype == torch.float32:
+        return CSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _req(t, name, dtype=None, ndim=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    return t
+
+
+def csa_workspace_size(p: Params, op: int, B: int, Tq: int, n_max: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_load().csa_workspace_size(ctypes.byref(p.c()), op, B, Tq, n_max, ctypes.byref(n)))
+    return int(n.value)
+
+
+def csa_compress(p: Params, x, gate, kv_cmp_out, kv_raw_rot_out=None, stream=None):
+    """x, gate [B][T][d] -> kv_cmp_out [B][N][d] (+ kv_raw_rot_out [B][T][d])."""
+    _req(x, "x", ndim=3)
+    _req(gate, "gate", x.dtype, 3)
+    _req(kv_cmp_out, "kv_cmp_out", x.dtype, 3)
+    if kv_raw_rot_out is not None:
+        _req(kv_raw_rot_out, "kv_raw_rot_out", x.dtype, 3)
+    B, T, d = x.shape
+    _check(_load().csa_compress(ctypes.byref(p.c()), _dtype_code(x), _ptr(x), _ptr(gate), B, T,
+                                _ptr(kv_cmp_out), _ptr(kv_raw_rot_out), _stream(stream)))
+
+
+def csa_index_scores(p: Params, q_idx, w, k_idx, q_pos, n_cmp, scores, stream=None):
+    """q_idx [B][Tq][H_I][d_I], w [B][Tq][H_I], k_idx [B][n_max][d_I] -> scores [B][Tq][n_max]."""
+    import torch
+    _req(q_idx, "q_idx", ndim=4)
+    _req(w, "w", torch.float32, 3)
+    _req(k_idx, "k_idx", q_idx.dtype, 3)
+    _req(q_pos, "q_pos", torch.int32, 2)
+    _req(n_cmp, "n_cmp", torch.int32, 1)
+    _req(scores, "scores", torch.float32, 3)
+    B, Tq = q_pos.shape
+    n_max = k_idx.shape[1]
+    _check(_load().csa_index_scores(ctypes.byref(p.c()), _dtype_code(q_idx), _ptr(q_idx), _ptr(w),
+                                    _ptr(k_idx), _ptr(q_pos), _ptr(n_cmp), B, Tq, n_max,
+                                    _ptr(scores), _stream(stream)))
+
+
+def csa_topk_select(p: Params, scores, q_pos, n_cmp, idx_out, ws=None, stream=None):
+    """scores [B][Tq][n_max] fp32 -> idx_out [B][Tq][topk] int32."""
+    import torch
+    _req(scores, "scores", torch.float32, 3)
+    _req(q_pos, "q_pos", torch.int32, 2)
+    _req(n_cmp, "n_cmp", torch.int32, 1)
+    _req(idx_out, "idx_out", torch.int32, 3)
+    B, Tq, n_max = scores.shape
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().csa_topk_select(ctypes.byref(p.c()), _ptr(scores), _ptr(q_pos), _ptr(n_cmp),
+                                   B, Tq, n_max, _ptr(idx_out), _ptr(ws), nb, _stream(stream)))
+
+
+def csa_index_topk(p: Params, q_idx, w, k_idx, q_pos, n_cmp, idx_out, ws, stream=None):
+    """Indexer + top-k; ws: csa_workspace_size(CSA_OP_INDEX_TOPK) bytes."""
+    import torch
+    _req(q_idx, "q_idx", ndim=4)
+    _req(w, "w", torch.float32, 3)
+    _req(k_idx, "k_idx", q_idx.dtype, 3)
+    _req(q_pos, "q_pos", torch.int32, 2)
+    _req(n_cmp, "n_cmp", torch.int32, 1)
+    _req(idx_out, "idx_out", torch.int32, 3)
+    B, Tq = q_pos.shape
+    n_max = k_idx.shape[1]
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().csa_index_topk(ctypes.byref(p.c()), _dtype_code(q_idx), _ptr(q_idx), _ptr(w),
+                                  _ptr(k_idx), _ptr(q_pos), _ptr(n_cmp), B, Tq, n_max,
+                                  _ptr(idx_out), _ptr(ws), nb, _stream(stream)))
+
+
+def _attn(fn, p, q, q_pos, kv_cmp, sel, kv_raw, raw_pos0, n_raw, sink, out, ws, stream):
+    import torch
+    _req(q, "q", ndim=4)
+    _req(q_pos, "q_pos", torch.int32, 2)
+    _req(kv_cmp, "kv_cmp", q.dtype, 3)
+    _req(kv_raw, "kv_raw", q.dtype, 3)
+    _req(raw_pos0, "raw_pos0", torch.int32, 1)
+    _req(n_raw, "n_raw", torch.int32, 1)
+    _req(sink, "sink", torch.float32, 1)
+    _req(out, "out", q.dtype, 4)
+    B, Tq = q_pos.shape
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(fn(ctypes.byref(p.c()), _dtype_code(q), _ptr(q), _ptr(q_pos), _ptr(kv_cmp), _ptr(sel),
+              kv_cmp.shape[1], _ptr(kv_raw), _ptr(raw_pos0), _ptr(n_raw), kv_raw.shape[1],
+              _ptr(sink), B, Tq, _ptr(out), _ptr(ws), nb, _stream(stream)))
+
+
+def csa_sparse_attn(p: Params, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out,
+                    ws=None, stream=None):
+    """q [B][Tq][H][d], idx [B][Tq][topk] -> out [B][Tq][H][d]."""
+    import torch
+    _req(idx, "idx", torch.int32, 3)
+    _attn(_load().csa_sparse_attn, p, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out,
+          ws, stream)
+
+
+def hca_attn(p: Params, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, out, ws=None,
+             stream=None):
+    """Dense attention over every visible entry + window."""
+    import torch
+    _req(n_cmp, "n_cmp", torch.int32, 1)
+    _attn(_load().hca_attn, p, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, out, ws,
+          stream)
+
+
+def csa_poll_device_error(stream=None):
+    _check(_load().csa_poll_device_error(_stream(stream)))

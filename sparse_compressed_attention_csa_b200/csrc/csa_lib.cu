@@ -1,0 +1,401 @@
+// C ABI of the CSA library: argument validation, workspace sizing and kernel
+// launches.  Declarations and the contract of every call are in csa.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "attn_simt.cuh"
+#include "common.cuh"
+#include "compress.cuh"
+#include "csa.h"
+#include "indexer_simt.cuh"
+#include "topk.cuh"
+
+namespace csa {
+namespace {
+
+thread_local char g_detail[512] = "";
+
+csa_status_t fail(csa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+csa_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(CSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define CSA_CHECK(expr)                  \
+  do {                                   \
+    csa_status_t _s = (expr);            \
+    if (_s != CSA_OK) return _s;         \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+csa_status_t check_ptr(const void* p, const char* name, bool nullable = false) {
+  if (p == nullptr) {
+    if (nullable) return CSA_OK;
+    return fail(CSA_ERR_INVALID_ARGUMENT, "%s is NULL", name);
+  }
+  if (!aligned16(p)) return fail(CSA_ERR_MISALIGNED, "%s is not 16-byte aligned", name);
+  return CSA_OK;
+}
+
+csa_status_t check_device() {
+  static int checked[64];  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev >= 0 && dev < 64 && checked[dev] == 1) return CSA_OK;
+  int major = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (major != 10) {
+    if (dev >= 0 && dev < 64) checked[dev] = 2;
+    return fail(CSA_ERR_UNSUPPORTED_DEVICE, "device %d is sm_%d0, the library is built for sm_100a",
+                dev, major);
+  }
+  if (dev >= 0 && dev < 64) checked[dev] = 1;
+  return CSA_OK;
+}
+
+csa_status_t check_params(const csa_params_t* p) {
+  if (p == nullptr) return fail(CSA_ERR_INVALID_ARGUMENT, "params is NULL");
+  if (p->d != 64 && p->d != 128 && p->d != 256 && p->d != 512 && p->d != 1024)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "d=%d: supported 64, 128, 256, 512, 1024", p->d);
+  if (p->rope_dim < 0 || p->rope_dim > p->d || (p->rope_dim & 1) || ((p->d - p->rope_dim) & 31))
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE,
+                "rope_dim=%d: must be even, <= d and leave a multiple of 32 unrotated dims",
+                p->rope_dim);
+  if (!(p->theta > 0.f) || !std::isfinite(p->theta))
+    return fail(CSA_ERR_INVALID_ARGUMENT, "theta must be positive and finite");
+  if (!std::isfinite(p->scale)) return fail(CSA_ERR_INVALID_ARGUMENT, "scale must be finite");
+  if (p->n_heads < 1 || p->n_heads > 65535)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "n_heads=%d out of [1, 65535]", p->n_heads);
+  if (p->width < 1 || p->stride < 1)
+    return fail(CSA_ERR_INVALID_ARGUMENT, "width=%d stride=%d must be >= 1", p->width, p->stride);
+  if (p->window < 0) return fail(CSA_ERR_INVALID_ARGUMENT, "window=%d < 0", p->window);
+  return CSA_OK;
+}
+
+csa_status_t check_indexer_shape(const csa_params_t* p) {
+  if (p->idx_heads < 1 || p->idx_dim < 2 || (p->idx_dim & 1) ||
+      p->idx_heads * p->idx_dim > 16384)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE,
+                "idx_heads=%d idx_dim=%d: need idx_dim even and idx_heads*idx_dim <= 16384",
+                p->idx_heads, p->idx_dim);
+  return CSA_OK;
+}
+
+csa_status_t check_topk(const csa_params_t* p) {
+  if (p->topk < 1 || p->topk > (1 << 20))
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "topk=%d out of [1, 2^20]", p->topk);
+  return CSA_OK;
+}
+
+csa_status_t check_dtype(csa_dtype_t dt) {
+  if (dt != CSA_F32 && dt != CSA_BF16) return fail(CSA_ERR_INVALID_ARGUMENT, "bad dtype %d", dt);
+  return CSA_OK;
+}
+
+csa_status_t check_sizes(int B, int Tq, int n_max) {
+  if (B < 1 || Tq < 1 || n_max < 0 || B > 65535 || Tq > 65535)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "B=%d Tq=%d n_max=%d out of range", B, Tq, n_max);
+  return CSA_OK;
+}
+
+csa_status_t launched(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return CSA_OK;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t scores_bytes(int B, int Tq, int n_max) {
+  return round_up((size_t)B * Tq * (size_t)n_max * sizeof(float), 256);
+}
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+#define CSA_API extern "C" __attribute__((visibility("default")))
+
+CSA_API int csa_abi_version(void) { return CSA_ABI_VERSION; }
+
+CSA_API const char* csa_status_string(csa_status_t s) {
+  switch (s) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARGUMENT: return "CSA_ERR_INVALID_ARGUMENT";
+    case CSA_ERR_MISALIGNED: return "CSA_ERR_MISALIGNED";
+    case CSA_ERR_UNSUPPORTED_SHAPE: return "CSA_ERR_UNSUPPORTED_SHAPE";
+    case CSA_ERR_UNSUPPORTED_DEVICE: return "CSA_ERR_UNSUPPORTED_DEVICE";
+    case CSA_ERR_WORKSPACE_TOO_SMALL: return "CSA_ERR_WORKSPACE_TOO_SMALL";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    case CSA_ERR_DEVICE_TIMEOUT: return "CSA_ERR_DEVICE_TIMEOUT";
+    case CSA_ERR_DEVICE_BOUNDS: return "CSA_ERR_DEVICE_BOUNDS";
+  }
+  return "CSA_ERR_UNKNOWN";
+}
+
+CSA_API const char* csa_last_error_detail(void) { return g_detail; }
+
+CSA_API csa_status_t csa_workspace_size(const csa_params_t* p, csa_op_t op, int32_t B, int32_t Tq,
+                                int32_t n_max, size_t* bytes) {
+  if (bytes == nullptr) return fail(CSA_ERR_INVALID_ARGUMENT, "bytes is NULL");
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_sizes(B, Tq, n_max));
+  switch (op) {
+    case CSA_OP_COMPRESS: *bytes = 0; return CSA_OK;
+    case CSA_OP_TOPK_SELECT: *bytes = 0; return CSA_OK;
+    case CSA_OP_INDEX_TOPK: *bytes = scores_bytes(B, Tq, n_max); return CSA_OK;
+    case CSA_OP_SPARSE_ATTN: *bytes = 0; return CSA_OK;
+    case CSA_OP_HCA_ATTN: *bytes = 0; return CSA_OK;
+  }
+  return fail(CSA_ERR_INVALID_ARGUMENT, "bad op %d", (int)op);
+}
+
+CSA_API csa_status_t csa_compress(const csa_params_t* p, csa_dtype_t dtype, const void* x,
+                          const void* gate, int32_t B, int32_t T, void* kv_cmp_out,
+                          void* kv_raw_rot_out, void* stream) {
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_dtype(dtype));
+  CSA_CHECK(check_ptr(x, "x"));
+  CSA_CHECK(check_ptr(gate, "gate"));
+  CSA_CHECK(check_ptr(kv_raw_rot_out, "kv_raw_rot_out", true));
+  if (B < 1 || B > 65535 || T < 0) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "B=%d T=%d", B, T);
+  const int N = T < p->width ? 0 : (T - p->width) / p->stride + 1;
+  if (N > 0) CSA_CHECK(check_ptr(kv_cmp_out, "kv_cmp_out"));
+  CSA_CHECK(check_device());
+  const long long rows = (long long)N + (kv_raw_rot_out ? T : 0);
+  if (rows == 0) return CSA_OK;
+  if (rows > 2147483647LL) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "too many rows");
+  cudaStream_t s = (cudaStream_t)stream;
+  dim3 grid((unsigned)rows, (unsigned)B);
+  const int threads = p->d / 2 < 256 ? p->d / 2 : 256;
+  if (dtype == CSA_BF16)
+    k_compress<__nv_bfloat16><<<grid, threads, 0, s>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)gate, T, p->d, N, p->width, p->stride,
+        p->rope_dim, (double)p->theta, p->pos_offset, (__nv_bfloat16*)kv_cmp_out,
+        (__nv_bfloat16*)kv_raw_rot_out);
+  else
+    k_compress<float><<<grid, threads, 0, s>>>((const float*)x, (const float*)gate, T, p->d, N,
+                                               p->width, p->stride, p->rope_dim,
+                                               (double)p->theta, p->pos_offset,
+                                               (float*)kv_cmp_out, (float*)kv_raw_rot_out);
+  return launched("k_compress");
+}
+
+static csa_status_t index_scores_impl(const csa_params_t* p, csa_dtype_t dtype, const void* q_idx,
+                                      const float* w, const void* k_idx, const int32_t* q_pos,
+                                      const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
+                                      float* scores, cudaStream_t s) {
+  if (n_max == 0) return CSA_OK;
+  const int H_I = p->idx_heads, d_I = p->idx_dim;
+  dim3 grid((unsigned)((n_max + kIdxSimtKeys - 1) / kIdxSimtKeys), (unsigned)Tq, (unsigned)B);
+  const size_t smem = (size_t)(H_I * d_I + H_I) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e;
+    if (dtype == CSA_BF16)
+      e = cudaFuncSetAttribute(k_index_scores_simt<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    else
+      e = cudaFuncSetAttribute(k_index_scores_simt<float>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_index_scores_simt)");
+  }
+  if (dtype == CSA_BF16)
+    k_index_scores_simt<__nv_bfloat16><<<grid, kIdxSimtKeys, smem, s>>>(
+        (const __nv_bfloat16*)q_idx, w, (const __nv_bfloat16*)k_idx, q_pos, n_cmp, Tq, n_max,
+        H_I, d_I, p->width, p->stride, scores);
+  else
+    k_index_scores_simt<float><<<grid, kIdxSimtKeys, smem, s>>>(
+        (const float*)q_idx, w, (const float*)k_idx, q_pos, n_cmp, Tq, n_max, H_I, d_I,
+        p->width, p->stride, scores);
+  return launched("k_index_scores_simt");
+}
+
+static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const int32_t* q_pos,
+                              const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
+                              int32_t* idx_out, cudaStream_t s) {
+  const unsigned rows = (unsigned)B * (unsigned)Tq;
+  if (n_max >= 8192)
+    k_topk_rows<1024><<<rows, 1024, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, p->topk, p->width,
+                                            p->stride, idx_out);
+  else
+    k_topk_rows<256><<<rows, 256, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, p->topk, p->width,
+                                          p->stride, idx_out);
+  return launched("k_topk_rows");
+}
+
+CSA_API csa_status_t csa_index_scores(const csa_params_t* p, csa_dtype_t dtype, const void* q_idx,
+                              const float* w, const void* k_idx, const int32_t* q_pos,
+                              const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
+                              float* scores, void* stream) {
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_dtype(dtype));
+  CSA_CHECK(check_indexer_shape(p));
+  CSA_CHECK(check_sizes(B, Tq, n_max));
+  CSA_CHECK(check_ptr(q_idx, "q_idx"));
+  CSA_CHECK(check_ptr(w, "w"));
+  CSA_CHECK(check_ptr(k_idx, "k_idx", n_max == 0));
+  CSA_CHECK(check_ptr(q_pos, "q_pos"));
+  CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
+  CSA_CHECK(check_ptr(scores, "scores", n_max == 0));
+  CSA_CHECK(check_device());
+  return index_scores_impl(p, dtype, q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, scores,
+                           (cudaStream_t)stream);
+}
+
+CSA_API csa_status_t csa_topk_select(const csa_params_t* p, const float* scores, const int32_t* q_pos,
+                             const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
+                             int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_topk(p));
+  CSA_CHECK(check_sizes(B, Tq, n_max));
+  CSA_CHECK(check_ptr(scores, "scores", n_max == 0));
+  CSA_CHECK(check_ptr(q_pos, "q_pos"));
+  CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
+  CSA_CHECK(check_ptr(idx_out, "idx_out"));
+  CSA_CHECK(check_ptr(ws, "ws", true));
+  (void)ws_bytes;
+  CSA_CHECK(check_device());
+  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, (cudaStream_t)stream);
+}
+
+CSA_API csa_status_t csa_index_topk(const csa_params_t* p, csa_dtype_t dtype, const void* q_idx,
+                            const float* w, const void* k_idx, const int32_t* q_pos,
+                            const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
+                            int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_dtype(dtype));
+  CSA_CHECK(check_indexer_shape(p));
+  CSA_CHECK(check_topk(p));
+  CSA_CHECK(check_sizes(B, Tq, n_max));
+  CSA_CHECK(check_ptr(q_idx, "q_idx"));
+  CSA_CHECK(check_ptr(w, "w"));
+  CSA_CHECK(check_ptr(k_idx, "k_idx", n_max == 0));
+  CSA_CHECK(check_ptr(q_pos, "q_pos"));
+  CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
+  CSA_CHECK(check_ptr(idx_out, "idx_out"));
+  const size_t need = scores_bytes(B, Tq, n_max);
+  if (need > 0) CSA_CHECK(check_ptr(ws, "ws"));
+  if (ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes, need %zu", ws_bytes, need);
+  CSA_CHECK(check_device());
+  cudaStream_t s = (cudaStream_t)stream;
+  float* scores = (float*)ws;
+  CSA_CHECK(index_scores_impl(p, dtype, q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, scores, s));
+  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, s);
+}
+
+static csa_status_t attn_common_checks(const csa_params_t* p, csa_dtype_t dtype, const void* q,
+                                       const int32_t* q_pos, const void* kv_cmp, int32_t n_max,
+                                       const void* kv_raw, const int32_t* raw_pos0,
+                                       const int32_t* n_raw, int32_t raw_max, const float* sink,
+                                       int32_t B, int32_t Tq, void* out) {
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_dtype(dtype));
+  CSA_CHECK(check_sizes(B, Tq, n_max));
+  if (raw_max < 0) return fail(CSA_ERR_INVALID_ARGUMENT, "raw_max=%d < 0", raw_max);
+  CSA_CHECK(check_ptr(q, "q"));
+  CSA_CHECK(check_ptr(q_pos, "q_pos"));
+  CSA_CHECK(check_ptr(kv_cmp, "kv_cmp", n_max == 0));
+  CSA_CHECK(check_ptr(kv_raw, "kv_raw", raw_max == 0));
+  CSA_CHECK(check_ptr(raw_pos0, "raw_pos0"));
+  CSA_CHECK(check_ptr(n_raw, "n_raw"));
+  CSA_CHECK(check_ptr(sink, "sink"));
+  return check_ptr(out, "out");
+}
+
+template <bool kHca>
+static csa_status_t launch_attn_simt(const AttnArgs& a, csa_dtype_t dtype, cudaStream_t s) {
+  dim3 grid((unsigned)a.H, (unsigned)a.Tq, (unsigned)a.B);
+  const int nk = a.d / 32;
+#define CSA_ATTN_CASE(NKV)                                                        \
+  case NKV:                                                                       \
+    if (dtype == CSA_BF16)                                                        \
+      k_attn_simt<__nv_bfloat16, kHca, NKV><<<grid, 32 * kAttnSimtWarps, 0, s>>>(a); \
+    else                                                                          \
+      k_attn_simt<float, kHca, NKV><<<grid, 32 * kAttnSimtWarps, 0, s>>>(a);      \
+    break;
+  switch (nk) {
+    CSA_ATTN_CASE(2)
+    CSA_ATTN_CASE(4)
+    CSA_ATTN_CASE(8)
+    CSA_ATTN_CASE(16)
+    CSA_ATTN_CASE(32)
+    default: return fail(CSA_ERR_UNSUPPORTED_SHAPE, "d=%d", a.d);
+  }
+#undef CSA_ATTN_CASE
+  return launched("k_attn_simt");
+}
+
+static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32_t* q_pos,
+                               const void* kv_cmp, const int32_t* idx, const int32_t* n_cmp,
+                               int32_t n_max, const void* kv_raw, const int32_t* raw_pos0,
+                               const int32_t* n_raw, int32_t raw_max, const float* sink,
+                               int32_t B, int32_t Tq, void* out) {
+  AttnArgs a;
+  a.q = q; a.q_pos = q_pos; a.kv_cmp = kv_cmp; a.idx = idx; a.n_cmp = n_cmp; a.n_max = n_max;
+  a.kv_raw = kv_raw; a.raw_pos0 = raw_pos0; a.n_raw = n_raw; a.raw_max = raw_max; a.sink = sink;
+  a.B = B; a.Tq = Tq; a.H = p->n_heads; a.d = p->d; a.rope_dim = p->rope_dim; a.topk = p->topk;
+  a.window = p->window; a.width = p->width; a.stride = p->stride; a.scale = p->scale;
+  a.theta = (double)p->theta; a.out = out;
+  return a;
+}
+
+CSA_API csa_status_t csa_sparse_attn(const csa_params_t* p, csa_dtype_t dtype, const void* q,
+                             const int32_t* q_pos, const void* kv_cmp, const int32_t* idx,
+                             int32_t n_max, const void* kv_raw, const int32_t* raw_pos0,
+                             const int32_t* n_raw, int32_t raw_max, const float* sink,
+                             int32_t B, int32_t Tq, void* out, void* ws, size_t ws_bytes,
+                             void* stream) {
+  CSA_CHECK(attn_common_checks(p, dtype, q, q_pos, kv_cmp, n_max, kv_raw, raw_pos0, n_raw,
+                               raw_max, sink, B, Tq, out));
+  CSA_CHECK(check_topk(p));
+  CSA_CHECK(check_ptr(idx, "idx"));
+  CSA_CHECK(check_device());
+  (void)ws; (void)ws_bytes;
+  AttnArgs a = make_attn_args(p, q, q_pos, kv_cmp, idx, nullptr, n_max, kv_raw, raw_pos0, n_raw,
+                              raw_max, sink, B, Tq, out);
+  return launch_attn_simt<false>(a, dtype, (cudaStream_t)stream);
+}
+
+CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const void* q,
+                      const int32_t* q_pos, const void* kv_cmp, const int32_t* n_cmp,
+                      int32_t n_max, const void* kv_raw, const int32_t* raw_pos0,
+                      const int32_t* n_raw, int32_t raw_max, const float* sink, int32_t B,
+                      int32_t Tq, void* out, void* ws, size_t ws_bytes, void* stream) {
+  CSA_CHECK(attn_common_checks(p, dtype, q, q_pos, kv_cmp, n_max, kv_raw, raw_pos0, n_raw,
+                               raw_max, sink, B, Tq, out));
+  CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
+  CSA_CHECK(check_device());
+  (void)ws; (void)ws_bytes;
+  AttnArgs a = make_attn_args(p, q, q_pos, kv_cmp, nullptr, n_cmp, n_max, kv_raw, raw_pos0,
+                              n_raw, raw_max, sink, B, Tq, out);
+  return launch_attn_simt<true>(a, dtype, (cudaStream_t)stream);
+}
+
+CSA_API csa_status_t csa_poll_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (v == 0) return CSA_OK;
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  return fail((csa_status_t)v, "device reported %s", csa_status_string((csa_status_t)v));
+}
+

@@ -1,0 +1,75 @@
+"""User-level entry points: allocate outputs and workspace with torch, then
+call the C ABI.  Every step runs in the CUDA library.
+
+    decode: csa_decode(p, q, q_idx, w, k_idx, kv_cmp, kv_raw, ...) -> (idx, out)
+    prefill: csa_prefill(p, x, gate, q_idx, w, k_idx, q, sink) -> (kv_cmp, kv_raw, idx, out)
+    HCA decode: hca_decode(p, q, kv_cmp, kv_raw, ...) -> out
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+class Workspace:
+    """A reusable device scratch buffer that grows on demand."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int):
+        if nbytes == 0:
+            return None
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+
+def csa_decode(p: L.Params, q, q_pos, q_idx, w, k_idx, n_cmp, kv_cmp, kv_raw, raw_pos0, n_raw,
+               sink, ws: Workspace | None = None, idx=None, out=None, stream=None):
+    """Indexer + top-k + sparse attention for Tq query tokens per sequence."""
+    ws = ws or Workspace(q.device)
+    B, Tq = q_pos.shape
+    n_max = k_idx.shape[1]
+    if idx is None:
+        idx = torch.empty((B, Tq, p.topk), dtype=torch.int32, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    nb = L.csa_workspace_size(p, L.CSA_OP_INDEX_TOPK, B, Tq, n_max)
+    L.csa_index_topk(p, q_idx, w, k_idx, q_pos, n_cmp, idx, ws.get(nb), stream)
+    nb = L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, B, Tq, kv_cmp.shape[1])
+    L.csa_sparse_attn(p, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out, ws.get(nb),
+                      stream)
+    return idx, out
+
+
+def csa_prefill(p: L.Params, x, gate, q_idx, w, k_idx, q, sink, ws: Workspace | None = None,
+                stream=None):
+    """The whole layer on B sequences of T tokens, every token a causal query."""
+    ws = ws or Workspace(x.device)
+    B, T, d = x.shape
+    N = 0 if T < p.width else (T - p.width) // p.stride + 1
+    dev = x.device
+    kv_cmp = torch.empty((B, N, d), dtype=x.dtype, device=dev)
+    kv_raw = torch.empty((B, T, d), dtype=x.dtype, device=dev)
+    L.csa_compress(p, x, gate, kv_cmp, kv_raw, stream)
+    q_pos = torch.arange(T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+    n_cmp = torch.full((B,), N, dtype=torch.int32, device=dev)
+    raw_pos0 = torch.zeros((B,), dtype=torch.int32, device=dev)
+    n_raw = torch.full((B,), T, dtype=torch.int32, device=dev)
+    idx, out = csa_decode(p, q, q_pos, q_idx, w, k_idx, n_cmp, kv_cmp, kv_raw, raw_pos0, n_raw,
+                          sink, ws, stream=stream)
+    return kv_cmp, kv_raw, idx, out
+
+
+def hca_decode(p: L.Params, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink,
+               ws: Workspace | None = None, out=None, stream=None):
+    ws = ws or Workspace(q.device)
+    B, Tq = q_pos.shape
+    if out is None:
+        out = torch.empty_like(q)
+    nb = L.csa_workspace_size(p, L.CSA_OP_HCA_ATTN, B, Tq, kv_cmp.shape[1])
+    L.hca_attn(p, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, out, ws.get(nb), stream)
+    return out

@@ -1,0 +1,218 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Bit-exact top-k indices (and indexer scores, which are exact integers times
+powers of two); outputs within max-abs / relative-L2 bounds (bf16 2e-2 /
+5e-3, fp32 1e-5).  Every workload runs at its full size in the launch
+configuration the benchmark times; the oracle checks every sequence of the
+decode workloads and a stratified sample of the prefill queries.  Smaller
+cases cover several tiles with ragged tails and the edge cases.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_close, dev, f64, host64, params_of, run_decode, run_hca, run_prefill
+from sparse_compressed_attention_csa_b200 import (CsaError, Params, csa_compress,
+                                                  csa_index_scores, csa_poll_device_error,
+                                                  csa_sparse_attn, csa_topk_select, layer)
+from sparse_compressed_attention_csa_b200 import workloads as W
+from sparse_compressed_attention_csa_b200.workloads import bits_to_f32, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _vals(a):
+    """Generated array as real values (fp32 view of bf16 bits)."""
+    return bits_to_f32(a) if a.dtype == np.uint16 else a
+
+
+# ------------------------------------------------------------------ oracle drivers
+def oracle_decode(wl, data, seqs):
+    idx_all, out_all = [], []
+    for b in seqs:
+        qp = data["q_pos"][b]
+        idx = oracle.index_topk(f64(data, "q_idx", b), data["w"][b], f64(data, "k_idx", b), qp,
+                                int(data["n_cmp"][b]), wl.width, wl.stride, wl.topk)
+        out = oracle.sparse_attn(f64(data, "q", b), qp, _vals(data["kv_cmp"][b]), idx,
+                                 _vals(data["kv_raw"][b]), int(data["raw_pos0"][b]),
+                                 int(data["n_raw"][b]), data["sink"], wl.scale, wl.window,
+                                 wl.rope_dim, wl.theta)
+        idx_all.append(idx)
+        out_all.append(out)
+    return np.stack(idx_all), np.stack(out_all)
+
+
+def check_decode(wl, seqs=None):
+    data = W.generate(wl)
+    idx, out = run_decode(wl, data)
+    seqs = list(range(wl.B)) if seqs is None else seqs
+    idx_o, out_o = oracle_decode(wl, data, seqs)
+    got_idx = idx.cpu().numpy()[seqs]
+    assert np.array_equal(got_idx, idx_o), "top-k indices differ"
+    assert_close(host64(out)[seqs], out_o, wl.dtype, wl.name)
+
+
+def check_hca(wl, seqs=None):
+    data = W.generate(wl)
+    out = run_hca(wl, data)
+    seqs = list(range(wl.B)) if seqs is None else seqs
+    got = host64(out)[seqs]
+    want = np.stack([oracle.hca_attn(f64(data, "q", b), data["q_pos"][b],
+                                     _vals(data["kv_cmp"][b]), int(data["n_cmp"][b]),
+                                     _vals(data["kv_raw"][b]), int(data["raw_pos0"][b]),
+                                     int(data["n_raw"][b]), data["sink"], wl.scale, wl.window,
+                                     wl.width, wl.stride, wl.rope_dim, wl.theta)
+                     for b in seqs])
+    assert_close(got, want, wl.dtype, wl.name)
+
+
+def check_prefill(wl, rows=None):
+    data = W.generate(wl)
+    kv_cmp, kv_raw, idx, out = run_prefill(wl, data)
+    T = wl.T
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    for b in range(wl.B):
+        x, g = f64(data, "x", b), f64(data, "g", b)
+        cmp_o = oracle.compress(x, g, wl.width, wl.stride, wl.rope_dim, wl.theta, wl.pos_offset)
+        assert_close(host64(kv_cmp[b]), cmp_o, wl.dtype, "compressed entries")
+        raw_o = oracle.rotate_raw(x, 0, wl.rope_dim, wl.theta)
+        assert_close(host64(kv_raw[b]), raw_o, wl.dtype, "rotated raw rows")
+        qp = data["q_pos"][b]
+        idx_o = oracle.index_topk(_vals(data["q_idx"][b]), data["w"][b], f64(data, "k_idx", b),
+                                  qp, cmp_o.shape[0], wl.width, wl.stride, wl.topk, rows)
+        assert np.array_equal(idx[b].cpu().numpy()[rows], idx_o), "top-k indices differ"
+        out_o = oracle.sparse_attn(to_f64(data["q"][b][rows]), qp[rows], cmp_o, idx_o, raw_o, 0,
+                                   T, data["sink"], wl.scale, wl.window, wl.rope_dim, wl.theta)
+        sel = torch.as_tensor(rows, device=out.device)
+        assert_close(host64(out[b][sel]), out_o, wl.dtype, wl.name)
+
+
+# ------------------------------------------------------------------ the five workloads
+def test_tiny_f32_full_layer():
+    check_prefill(W.TINY_F32)
+
+
+def test_csa_decode_64k_bs32():
+    check_decode(W.CSA_DECODE_64K)
+
+
+def test_csa_decode_1m_bs4():
+    check_decode(W.CSA_DECODE_1M)
+
+
+def test_hca_decode_128k_bs16():
+    check_hca(W.HCA_DECODE_128K)
+
+
+def test_csa_prefill_8k():
+    rng = np.random.default_rng(1234)
+    rows = np.unique(np.concatenate([np.arange(0, 16), np.arange(4095, 4104),
+                                     np.arange(8176, 8192), rng.integers(0, 8192, 64)]))
+    check_prefill(W.CSA_PREFILL_8K, rows)
+
+
+# ------------------------------------------------------------------ smaller cases
+def test_decode_ragged_tiles():
+    # N = 1249 (ragged), selection active (n_vis > k), raw window 128
+    check_decode(W.CSA_DECODE_64K.replace(B=3, T=5003, seed=21))
+
+
+def test_decode_fewer_visible_than_k():
+    check_decode(W.CSA_DECODE_64K.replace(B=2, T=2100, seed=22))  # N = 524 < 1024
+
+
+def test_prefill_ragged_small():
+    check_prefill(W.CSA_PREFILL_8K.replace(T=777, topk=64, seed=23))
+
+
+def test_prefill_small_heads_f32():
+    check_prefill(W.TINY_F32.replace(T=203, n_heads=3, topk=7, window=5, seed=24, pos_offset=2))
+
+
+def test_hca_ragged_and_early_queries():
+    check_hca(W.HCA_DECODE_128K.replace(B=3, T=1000, seed=25))   # N = 7
+    check_hca(W.HCA_DECODE_128K.replace(B=2, T=100, seed=26))    # N = 0: window + sink only
+
+
+def test_compress_hca_width_bf16_and_f32():
+    for dtype in ("bf16", "f32"):
+        wl = W.CSA_PREFILL_8K.replace(dtype=dtype, T=1000, width=128, stride=128, seed=27)
+        data = W.generate(wl)
+        p = params_of(wl)
+        x, g = dev(data["x"]), dev(data["g"])
+        N = wl.n_cmp
+        kv = torch.empty((1, N, wl.d), dtype=x.dtype, device="cuda")
+        csa_compress(p, x, g, kv)
+        torch.cuda.synchronize()
+        want = oracle.compress(f64(data, "x", 0), f64(data, "g", 0), 128, 128, wl.rope_dim,
+                               wl.theta)
+        assert_close(host64(kv[0]), want, dtype, f"hca compress {dtype}")
+
+
+def test_index_scores_bit_exact():
+    wl = W.CSA_PREFILL_8K.replace(T=1503, seed=28)
+    data = W.generate(wl)
+    p = params_of(wl)
+    t = {k: dev(data[k]) for k in ("q_idx", "w", "k_idx", "q_pos", "n_cmp")}
+    sc = torch.full((1, wl.T, wl.n_cmp), float("nan"), dtype=torch.float32, device="cuda")
+    csa_index_scores(p, t["q_idx"], t["w"], t["k_idx"], t["q_pos"], t["n_cmp"], sc)
+    torch.cuda.synchronize()
+    got = sc[0].cpu().numpy().astype(np.float64)
+    want = oracle.index_scores(f64(data, "q_idx", 0), data["w"][0], f64(data, "k_idx", 0))
+    for tq in range(0, wl.T, 7):
+        nv = oracle.n_visible(tq, wl.n_cmp, wl.width, wl.stride)
+        assert np.array_equal(got[tq, :nv], want[tq, :nv]), tq
+
+
+def test_topk_select_adversarial_scores():
+    rng = np.random.default_rng(29)
+    n, k = 5000, 1024
+    cases = [
+        np.zeros(n),                                        # all tied
+        np.where(rng.random(n) < 0.5, 0.0, -0.0),           # signed zeros tie
+        rng.integers(0, 3, n).astype(np.float64),           # few distinct values
+        -rng.random(n),                                     # negatives
+        rng.standard_normal(n) * 1e-30,                     # tiny magnitudes
+        np.concatenate([np.full(n // 2, 7.0), rng.random(n - n // 2)]),
+        rng.standard_normal(n).astype(np.float32).astype(np.float64),
+    ]
+    scores = np.stack(cases).astype(np.float32)[:, None, :]     # [B, 1, n]
+    B = scores.shape[0]
+    p = Params(topk=k, width=8, stride=4)
+    q_pos = np.full((B, 1), 4 * (n - 1) + 7, dtype=np.int32)   # every entry visible
+    n_cmp = np.full((B,), n, dtype=np.int32)
+    idx = torch.empty((B, 1, k), dtype=torch.int32, device="cuda")
+    csa_topk_select(p, dev(scores), dev(q_pos), dev(n_cmp), idx)
+    torch.cuda.synchronize()
+    got = idx.cpu().numpy()
+    for b in range(B):
+        want = oracle.topk_select(scores[b, 0].astype(np.float64), n, k)
+        assert np.array_equal(got[b, 0], want), b
+
+
+def test_deterministic_repeat():
+    wl = W.CSA_DECODE_64K.replace(B=2, T=9000, seed=30)
+    data = W.generate(wl)
+    i1, o1 = run_decode(wl, data)
+    i2, o2 = run_decode(wl, data)
+    assert torch.equal(i1, i2)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+def test_device_bounds_error_is_reported():
+    """An index past the cache is skipped and reported, not dereferenced."""
+    wl = W.CSA_DECODE_64K.replace(B=1, T=600, seed=31, topk=16)
+    data = W.generate(wl)
+    p = params_of(wl)
+    t = {k: dev(v) for k, v in data.items()}
+    idx = torch.arange(16, dtype=torch.int32, device="cuda").view(1, 1, 16).contiguous()
+    idx[0, 0, 5] = wl.n_cmp + 1000
+    out = torch.empty_like(t["q"])
+    csa_poll_device_error()
+    csa_sparse_attn(p, t["q"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"],
+                    t["n_raw"], t["sink"], out)
+    with pytest.raises(CsaError) as ei:
+        csa_poll_device_error()
+    assert ei.value.status == 8
+    csa_poll_device_error()  # cleared
