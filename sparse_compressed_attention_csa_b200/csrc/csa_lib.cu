@@ -1,17 +1,21 @@
 // C ABI of the CSA library: argument validation, workspace sizing and kernel
 // launches.  Declarations and the contract of every call are in csa.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "attn_simt.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "csa.h"
 #include "indexer_simt.cuh"
+#include "indexer_tc.cuh"
 #include "topk.cuh"
 
 namespace csa {
@@ -119,6 +123,73 @@ csa_status_t launched(const char* what) {
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+int num_sms() {
+  static int cached[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+// Opt a kernel into `bytes` of dynamic shared memory, once per (kernel,
+// device).
+template <typename K>
+csa_status_t set_smem_attr(K* kernel, size_t bytes, const char* name) {
+  struct Entry {
+    const void* fn;
+    int dev;
+  };
+  static Entry done[256];
+  static int n_done = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].fn == (const void*)kernel && done[i].dev == dev) return CSA_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bytes);
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  if (n_done < 256) done[n_done++] = Entry{(const void*)kernel, dev};
+  return CSA_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// libcuda link dependency).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map over [rows][inner] row-major, box [box_rows][box_inner],
+// 128-byte swizzle (box_inner * 2 must be 128).
+csa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                            uint32_t box_inner, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return CSA_OK;
+}
+
 size_t scores_bytes(int B, int Tq, int n_max) {
   return round_up((size_t)B * Tq * (size_t)n_max * sizeof(float), 256);
 }
@@ -195,12 +266,42 @@ CSA_API csa_status_t csa_compress(const csa_params_t* p, csa_dtype_t dtype, cons
   return launched("k_compress");
 }
 
+template <int QPB, int STAGES>
+static csa_status_t launch_index_tc(const void* q_idx, const float* w, const void* k_idx,
+                                    const int32_t* q_pos, const int32_t* n_cmp, int32_t B,
+                                    int32_t Tq, int32_t n_max, int width, int stride,
+                                    float* scores, cudaStream_t s) {
+  CUtensorMap tk, tq;
+  CSA_CHECK(make_tmap_bf16(&tk, k_idx, kIdxTcDim, (uint64_t)B * n_max, 64, kIdxTcKeys));
+  CSA_CHECK(make_tmap_bf16(&tq, q_idx, kIdxTcDim, (uint64_t)B * Tq * kIdxTcHeads, 64,
+                           QPB * kIdxTcHeads));
+  const size_t smem = sizeof(IdxTcSmem<QPB, STAGES>) + 1024;
+  CSA_CHECK(set_smem_attr(k_index_scores_tc<QPB, STAGES>, smem, "k_index_scores_tc"));
+  const int qblocks = (Tq + QPB - 1) / QPB;
+  int chunks = 1;
+  if (qblocks * B < num_sms()) chunks = num_sms() / (qblocks * B);
+  dim3 grid((unsigned)(qblocks * chunks), (unsigned)B);
+  k_index_scores_tc<QPB, STAGES><<<grid, kIdxTcThreads, smem, s>>>(
+      tk, tq, w, q_pos, n_cmp, Tq, n_max, width, stride, chunks, scores);
+  return launched("k_index_scores_tc");
+}
+
 static csa_status_t index_scores_impl(const csa_params_t* p, csa_dtype_t dtype, const void* q_idx,
                                       const float* w, const void* k_idx, const int32_t* q_pos,
                                       const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
                                       float* scores, cudaStream_t s) {
   if (n_max == 0) return CSA_OK;
   const int H_I = p->idx_heads, d_I = p->idx_dim;
+  // tensor-core path: the measured indexer shape in bf16
+  if (dtype == CSA_BF16 && H_I == kIdxTcHeads && d_I == kIdxTcDim &&
+      (long long)B * n_max >= kIdxTcKeys) {
+    if (Tq == 1)
+      return launch_index_tc<1, 6>(q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, p->width,
+                                   p->stride, scores, s);
+    if ((long long)B * Tq >= 2)
+      return launch_index_tc<2, 2>(q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, p->width,
+                                   p->stride, scores, s);
+  }
   dim3 grid((unsigned)((n_max + kIdxSimtKeys - 1) / kIdxSimtKeys), (unsigned)Tq, (unsigned)B);
   const size_t smem = (size_t)(H_I * d_I + H_I) * sizeof(float);
   if (smem > 48 * 1024) {
