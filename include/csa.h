@@ -194,6 +194,29 @@ csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const void* q,
                       const int32_t* n_raw, int32_t raw_max, const float* sink, int32_t B,
                       int32_t Tq, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Indexer + top-k that allocates nothing: the same computation and
+ * arguments as csa_index_topk, without `ws`.  The pages have no counterpart
+ * of this call; it serves callers that cannot call cudaMalloc or hand out a
+ * workspace - a host that passes the library only its input and output
+ * buffers, an engine whose allocator has already reserved all device
+ * memory, or a latency-critical loop that cannot afford cudaMalloc's
+ * device-wide synchronization.
+ *   Scratch: a fixed array of 2^21 fp32 scores (8 MiB) compiled into the
+ *   library; every GPU that loads the library holds it until the process
+ *   exits.  B * Tq * n_max above 2^21 returns CSA_ERR_UNSUPPORTED_SHAPE.
+ *   Nothing in the array needs clearing: each call writes every score it
+ *   reads.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture.
+ *   Every call shares the one array: calls whose work overlaps on the GPU
+ *   (different streams, or other host threads) race and give wrong indices.
+ *   Serialize them. */
+csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t dtype, const void* q_idx,
+                                    const float* w, const void* k_idx, const int32_t* q_pos,
+                                    const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
+                                    int32_t* idx_out, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the current device's error
  * word: CSA_OK, CSA_ERR_DEVICE_TIMEOUT or CSA_ERR_DEVICE_BOUNDS. */
 csa_status_t csa_poll_device_error(void* stream);

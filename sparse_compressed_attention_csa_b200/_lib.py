@@ -93,9 +93,12 @@ def _load():
     lib.csa_sparse_attn.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P,
                                     _I, _I, _P, _P, ctypes.c_size_t, _P]
     lib.hca_attn.argtypes = list(lib.csa_sparse_attn.argtypes)
+    lib.csa_index_topk_noalloc.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _P, _I, _I, _I, _P,
+                                           _P]
     lib.csa_poll_device_error.argtypes = [_P]
     for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
-              "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error"):
+              "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error",
+              "csa_index_topk_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -207,6 +210,24 @@ def csa_index_topk(p: Params, q_idx, w, k_idx, q_pos, n_cmp, idx_out, ws, stream
     _check(_load().csa_index_topk(ctypes.byref(p.c()), _dtype_code(q_idx), _ptr(q_idx), _ptr(w),
                                   _ptr(k_idx), _ptr(q_pos), _ptr(n_cmp), B, Tq, n_max,
                                   _ptr(idx_out), _ptr(ws), nb, _stream(stream)))
+
+
+def csa_index_topk_noalloc(p: Params, q_idx, w, k_idx, q_pos, n_cmp, idx_out, stream=None):
+    """Indexer + top-k without a workspace, for callers that cannot allocate
+    device memory.  Scores go to an 8 MiB array built into the library
+    (B * Tq * n_max <= 2**21); calls that overlap on the GPU share it and race."""
+    import torch
+    _req(q_idx, "q_idx", ndim=4)
+    _req(w, "w", torch.float32, 3)
+    _req(k_idx, "k_idx", q_idx.dtype, 3)
+    _req(q_pos, "q_pos", torch.int32, 2)
+    _req(n_cmp, "n_cmp", torch.int32, 1)
+    _req(idx_out, "idx_out", torch.int32, 3)
+    B, Tq = q_pos.shape
+    n_max = k_idx.shape[1]
+    _check(_load().csa_index_topk_noalloc(ctypes.byref(p.c()), _dtype_code(q_idx), _ptr(q_idx),
+                                          _ptr(w), _ptr(k_idx), _ptr(q_pos), _ptr(n_cmp), B, Tq,
+                                          n_max, _ptr(idx_out), _stream(stream)))
 
 
 def _attn(fn, p, q, q_pos, kv_cmp, sel, kv_raw, raw_pos0, n_raw, sink, out, ws, stream):

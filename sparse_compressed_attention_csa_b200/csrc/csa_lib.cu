@@ -487,6 +487,67 @@ CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const vo
   return launch_attn_simt<true>(a, dtype, (cudaStream_t)stream);
 }
 
+// ---------------------------------------------------------------------------
+// csa_index_topk_noalloc: the indexer + top-k for callers that cannot call
+// cudaMalloc (or hand out a workspace).  The scores live in the fixed
+// device array below instead of the caller's workspace.  Every GPU that
+// loads this library keeps the array (8 MiB) until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScoreFloats = size_t(1) << 21;  // B * Tq * n_max limit
+static __device__ __align__(256) float g_noalloc_scores[kNoAllocScoreFloats];
+
+// Device address of g_noalloc_scores on the current device.  In host code
+// the symbol's name is only a host-side stand-in, so the address is looked
+// up with cudaGetSymbolAddress once per device (the first call on a device)
+// and cached.
+static csa_status_t noalloc_scores_ptr(float** out) {
+  static float* ptrs[64];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(CSA_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scores);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    ptrs[dev] = static_cast<float*>(p);
+  }
+  *out = ptrs[dev];
+  return CSA_OK;
+}
+
+CSA_API csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t dtype,
+                                            const void* q_idx, const float* w, const void* k_idx,
+                                            const int32_t* q_pos, const int32_t* n_cmp,
+                                            int32_t B, int32_t Tq, int32_t n_max,
+                                            int32_t* idx_out, void* stream) {
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_dtype(dtype));
+  CSA_CHECK(check_indexer_shape(p));
+  CSA_CHECK(check_topk(p));
+  CSA_CHECK(check_sizes(B, Tq, n_max));
+  CSA_CHECK(check_ptr(q_idx, "q_idx"));
+  CSA_CHECK(check_ptr(w, "w"));
+  CSA_CHECK(check_ptr(k_idx, "k_idx", n_max == 0));
+  CSA_CHECK(check_ptr(q_pos, "q_pos"));
+  CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
+  CSA_CHECK(check_ptr(idx_out, "idx_out"));
+  const size_t need = (size_t)B * (size_t)Tq * (size_t)n_max;
+  if (need > kNoAllocScoreFloats)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE,
+                "B*Tq*n_max = %zu scores exceed the no-alloc scratch of %zu; use csa_index_topk "
+                "with a workspace",
+                need, kNoAllocScoreFloats);
+  CSA_CHECK(check_device());
+  float* scores = nullptr;
+  CSA_CHECK(noalloc_scores_ptr(&scores));
+  cudaStream_t s = (cudaStream_t)stream;
+  CSA_CHECK(index_scores_impl(p, dtype, q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, scores, s));
+  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, s);
+}
+
 CSA_API csa_status_t csa_poll_device_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
