@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "attn_simt.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "csa.h"
@@ -194,6 +195,38 @@ size_t scores_bytes(int B, int Tq, int n_max) {
   return round_up((size_t)B * Tq * (size_t)n_max * sizeof(float), 256);
 }
 
+int num_sms();
+
+// Tensor-core attention applies to the measured head shape in bf16.
+bool attn_tc_ok(const csa_params_t* p, csa_dtype_t dtype, bool hca, int n_max) {
+  if (dtype != CSA_BF16 || p->d != kAtDim || p->n_heads != kAtHeads) return false;
+  if (p->rope_dim > kAtDim) return false;
+  const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
+  return rows <= kAtRowCap;
+}
+
+// KV splits per query token: enough CTA pairs to cover the SMs, at least one
+// 64-row tile per split.
+int attn_splits(const csa_params_t* p, bool hca, int B, int Tq, int n_max) {
+  const long long units = (long long)B * Tq;
+  const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
+  long long s = num_sms() / (2 * units);
+  const long long max_s = (rows + kAtTile - 1) / kAtTile;
+  if (s > max_s) s = max_s;
+  if (s > 32) s = 32;
+  return s < 1 ? 1 : (int)s;
+}
+
+size_t attn_ws_bytes(const csa_params_t* p, csa_dtype_t dtype, bool hca, int B, int Tq,
+                     int n_max) {
+  if (!attn_tc_ok(p, dtype, hca, n_max)) return 0;
+  const int sp = attn_splits(p, hca, B, Tq, n_max);
+  if (sp == 1) return 0;
+  const size_t units = (size_t)B * Tq * sp * 2;
+  return round_up(units * kAtHeads * 256 * sizeof(float), 256) +
+         round_up(units * 2 * kAtHeads * sizeof(float), 256);
+}
+
 }  // namespace
 }  // namespace csa
 
@@ -229,8 +262,8 @@ CSA_API csa_status_t csa_workspace_size(const csa_params_t* p, csa_op_t op, int3
     case CSA_OP_COMPRESS: *bytes = 0; return CSA_OK;
     case CSA_OP_TOPK_SELECT: *bytes = 0; return CSA_OK;
     case CSA_OP_INDEX_TOPK: *bytes = scores_bytes(B, Tq, n_max); return CSA_OK;
-    case CSA_OP_SPARSE_ATTN: *bytes = 0; return CSA_OK;
-    case CSA_OP_HCA_ATTN: *bytes = 0; return CSA_OK;
+    case CSA_OP_SPARSE_ATTN: *bytes = attn_ws_bytes(p, CSA_BF16, false, B, Tq, n_max); return CSA_OK;
+    case CSA_OP_HCA_ATTN: *bytes = attn_ws_bytes(p, CSA_BF16, true, B, Tq, n_max); return CSA_OK;
   }
   return fail(CSA_ERR_INVALID_ARGUMENT, "bad op %d", (int)op);
 }
@@ -441,6 +474,57 @@ static csa_status_t launch_attn_simt(const AttnArgs& a, csa_dtype_t dtype, cudaS
   return launched("k_attn_simt");
 }
 
+template <bool kHca>
+static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, void* ws,
+                                   size_t ws_bytes, cudaStream_t s) {
+  const int sp = attn_splits(p, kHca, g.B, g.Tq, g.n_max);
+  const size_t need = attn_ws_bytes(p, CSA_BF16, kHca, g.B, g.Tq, g.n_max);
+  if (ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes, need %zu", ws_bytes, need);
+  if (need > 0) CSA_CHECK(check_ptr(ws, "ws"));
+  AttnTcArgs a;
+  a.q = (const __nv_bfloat16*)g.q;
+  a.q_pos = g.q_pos;
+  a.kv_cmp = (const __nv_bfloat16*)g.kv_cmp;
+  a.idx = g.idx;
+  a.n_cmp = g.n_cmp;
+  a.n_max = g.n_max;
+  a.kv_raw = (const __nv_bfloat16*)g.kv_raw;
+  a.raw_pos0 = g.raw_pos0;
+  a.n_raw = g.n_raw;
+  a.raw_max = g.raw_max;
+  a.sink = g.sink;
+  a.Tq = g.Tq;
+  a.topk = g.topk;
+  a.window = g.window;
+  a.width = g.width;
+  a.stride = g.stride;
+  a.rope_dim = g.rope_dim;
+  a.scale_log2 = g.scale * 1.4426950408889634f;
+  a.theta = g.theta;
+  a.splits = sp;
+  a.out = (__nv_bfloat16*)g.out;
+  a.part_o = nullptr;
+  a.part_ml = nullptr;
+  if (sp > 1) {
+    const size_t units = (size_t)g.B * g.Tq * sp * 2;
+    a.part_o = (float*)ws;
+    a.part_ml = (float*)((char*)ws + round_up(units * kAtHeads * 256 * sizeof(float), 256));
+  }
+  CUtensorMap tq;
+  CSA_CHECK(make_tmap_bf16(&tq, g.q, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
+  const size_t smem = sizeof(AtSmem) + 1024;
+  CSA_CHECK(set_smem_attr(k_attn_tc<kHca>, smem, "k_attn_tc"));
+  dim3 grid((unsigned)(2 * sp), (unsigned)(g.B * g.Tq));
+  k_attn_tc<kHca><<<grid, kAtThreads, smem, s>>>(a, tq);
+  CSA_CHECK(launched("k_attn_tc"));
+  if (sp > 1) {
+    k_attn_combine<<<dim3((unsigned)(g.B * g.Tq), 2, kAtHeads / 8), 256, 0, s>>>(a);
+    CSA_CHECK(launched("k_attn_combine"));
+  }
+  return CSA_OK;
+}
+
 static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32_t* q_pos,
                                const void* kv_cmp, const int32_t* idx, const int32_t* n_cmp,
                                int32_t n_max, const void* kv_raw, const int32_t* raw_pos0,
@@ -466,9 +550,10 @@ CSA_API csa_status_t csa_sparse_attn(const csa_params_t* p, csa_dtype_t dtype, c
   CSA_CHECK(check_topk(p));
   CSA_CHECK(check_ptr(idx, "idx"));
   CSA_CHECK(check_device());
-  (void)ws; (void)ws_bytes;
   AttnArgs a = make_attn_args(p, q, q_pos, kv_cmp, idx, nullptr, n_max, kv_raw, raw_pos0, n_raw,
                               raw_max, sink, B, Tq, out);
+  if (attn_tc_ok(p, dtype, false, n_max))
+    return launch_attn_tc<false>(p, a, ws, ws_bytes, (cudaStream_t)stream);
   return launch_attn_simt<false>(a, dtype, (cudaStream_t)stream);
 }
 
@@ -481,9 +566,10 @@ CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const vo
                                raw_max, sink, B, Tq, out));
   CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
   CSA_CHECK(check_device());
-  (void)ws; (void)ws_bytes;
   AttnArgs a = make_attn_args(p, q, q_pos, kv_cmp, nullptr, n_cmp, n_max, kv_raw, raw_pos0,
                               n_raw, raw_max, sink, B, Tq, out);
+  if (attn_tc_ok(p, dtype, true, n_max))
+    return launch_attn_tc<true>(p, a, ws, ws_bytes, (cudaStream_t)stream);
   return launch_attn_simt<true>(a, dtype, (cudaStream_t)stream);
 }
 

@@ -13,7 +13,8 @@ import torch
 
 import oracle
 from gpu_util import assert_close, dev, f64, host64, params_of, run_decode, run_hca, run_prefill
-from sparse_compressed_attention_csa_b200 import (CsaError, Params, csa_compress,
+from sparse_compressed_attention_csa_b200 import (CSA_OP_SPARSE_ATTN, CsaError, Params,
+                                                  csa_compress, csa_workspace_size,
                                                   csa_index_scores, csa_poll_device_error,
                                                   csa_sparse_attn, csa_topk_select, layer)
 from sparse_compressed_attention_csa_b200 import workloads as W
@@ -209,9 +210,11 @@ def test_device_bounds_error_is_reported():
     idx = torch.arange(16, dtype=torch.int32, device="cuda").view(1, 1, 16).contiguous()
     idx[0, 0, 5] = wl.n_cmp + 1000
     out = torch.empty_like(t["q"])
+    nb = csa_workspace_size(p, CSA_OP_SPARSE_ATTN, 1, 1, t["kv_cmp"].shape[1])
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
     csa_poll_device_error()
     csa_sparse_attn(p, t["q"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"],
-                    t["n_raw"], t["sink"], out)
+                    t["n_raw"], t["sink"], out, ws)
     with pytest.raises(CsaError) as ei:
         csa_poll_device_error()
     assert ei.value.status == 8
