@@ -5,28 +5,37 @@
 // Attention", "Partial RoPE" and "Output gate + sink" rows).
 //
 // One query token = one MMA M of 128 heads.  Its output O (128 x 512 fp32)
-// alone would fill all of TMEM (128 lanes x 512 columns), so every unit of
-// work is split in two CTAs by output dims: CTA `half` owns d_v columns
-// [256*half, 256*half + 256) and recomputes S = Q K^T itself.  Per CTA:
+// alone would fill all of TMEM (128 lanes x 512 columns), so each query is
+// split over NQ CTAs by output dims: CTA `part` owns d_v columns
+// [part * 512/NQ, (part + 1) * 512/NQ) and computes S = Q K^T itself.
 //
-//   TMEM  O_half [0,256) | S0 [256,320) | S1 [320,384) | Q_other [384,512)
-//   SMEM  Q_own (64 KB) | ring of 9 key/value chunks (16 KB each) | row list
+//   NQ = 2 (many queries: prefill; S recomputed twice)
+//     TMEM  O [0,256) | S0 [256,320) | S1 [320,384) | Q other half [384,512)
+//     SMEM  Q own half (64 KB) | ring of 9 chunks | row list
+//   NQ = 4 (few queries: decode; S recomputed four times, but the whole of Q
+//           sits in TMEM, which frees shared memory for a deeper gather ring)
+//     TMEM  O [0,128) | S0 [128,192) | S1 [192,256) | Q [256,512)
+//     SMEM  ring of 13 chunks | row list
 //
-// Q (rotated at the query position, rounded to bf16) is split by dims: the
-// CTA's own 256 dims sit in shared memory (SS MMAs), the other 256 in TMEM
-// (TS MMAs).  KV rows are gathered 64 at a time; each row is streamed as four
-// 128-dim chunks (16 B cp.async, 128B-swizzled).  The two chunks of the
-// other half feed only S and are released right after; the own two feed S
-// and then, as V, the PV product, and are held until it completes.
+// Q is rotated at the query position and rounded to bf16 once, after one TMA
+// load of [128 heads][64 dims] boxes.  KV rows are gathered 64 at a time by
+// 128 threads with 16-byte cp.async into 128B-swizzled shared memory (the
+// gather reaches full bandwidth only with many requests in flight, which
+// many issuing threads sustain and one-warp TMA gathers do not).  A row
+// streams as four 128-dim chunks through a FIFO ring; chunks outside the
+// CTA's output dims feed only S and are released right after it, the CTA's
+// own chunks then serve as V for the PV product and are held until it
+// completes.  The row list holds selected entries, then window rows, each
+// padded to a multiple of 4 with masked rows.
 //
 //   warp 8 (one thread): MMAs   S(i) = Q K_i^T  (N = 64, K = 512)
-//                               O   += P(i-1) V(i-1)  (A = P from TMEM, N = 2 x 128)
-//   warps 4-7: gather producers (cp.async, zero-filled tails)
+//                               O   += P(i-1) V(i-1)  (A = P from TMEM, N = 128 per chunk)
+//   warps 4-7: gather producers (q by TMA, rows by cp.async, no barriers)
 //   warps 0-3: one head per thread (= TMEM lane): online softmax in the
 //              log2 domain with a lazy rescale (only when the running max
 //              grows by more than 2^8), P written back over S as bf16,
 //              epilogue with the sink, the inverse output rotation and the
-//              store (or split-KV partials).
+//              store (or split-KV partials for k_attn_combine).
 // Every mbarrier wait is bounded; a timeout records CSA_ERR_DEVICE_TIMEOUT
 // and the CTA winds down, frees TMEM and exits.
 #pragma once
@@ -37,28 +46,14 @@ namespace csa {
 
 constexpr int kAtHeads = 128;
 constexpr int kAtDim = 512;
-constexpr int kAtTile = 64;          // KV rows per S tile (MMA N)
+constexpr int kAtTile = 64;                       // KV rows per S tile (MMA N)
 constexpr int kAtChunkBytes = kAtTile * 128 * 2;  // 64 rows x 128 dims bf16
-constexpr int kAtR1 = 3;             // ring of "other half" chunks
-constexpr int kAtR2 = 6;             // ring of "own half" chunks (V)
-constexpr int kAtRowCap = 2048;      // rows per query token (selected + window)
+constexpr int kAtSubBytes = kAtHeads * 128;       // q box: [128 heads][64 dims]
+constexpr int kAtRowCap = 2048;                   // rows per query token
+constexpr int kAtMaxRope = 128;                   // rotated dims supported
+constexpr int kAtMaxSlots = 13;
 constexpr int kAtThreads = 288;
 constexpr float kAtRescaleLog2 = 8.0f;
-
-struct AtSmem {
-  alignas(1024) uint8_t q_own[4][kAtHeads * 128];          // 4 x [128 heads][64 dims]
-  alignas(1024) uint8_t r1[kAtR1][kAtChunkBytes];          // [2][64 rows][128 B]
-  alignas(1024) uint8_t r2[kAtR2][kAtChunkBytes];
-  int rows[kAtRowCap];
-  const __nv_bfloat16* row_ptr[2][kAtTile];                // per tile parity
-  float cs[256], sn[256];
-  uint64_t r1_full[kAtR1], r1_empty[kAtR1], r2_full[kAtR2], r2_empty[kAtR2];
-  uint64_t s_full[2], p_full[2], pv_done[2], q_tma, q_ready, rows_ready;
-  uint32_t tmem_base;
-  int n_rows;
-  int abort_flag;
-  int prod_ok;
-};
 
 struct AttnTcArgs {
   const __nv_bfloat16* q;
@@ -74,12 +69,49 @@ struct AttnTcArgs {
   const float* sink;
   int Tq, topk, window, width, stride, rope_dim;
   float scale_log2;
-  double theta;
   int splits;
   __nv_bfloat16* out;  // splits == 1
-  float* part_o;       // splits > 1: [B*Tq][splits][2][128][256]
-  float* part_ml;      // [B*Tq][splits][2][2][128]  (m, l)
+  float* part_o;       // splits > 1: [B*Tq][splits][NQ][128][512/NQ]
+  float* part_ml;      // [B*Tq][splits][NQ][2][128]  (m, l)
+  double freq[kAtMaxRope / 2];  // RoPE frequencies theta^(-2i/rope_dim)
 };
+
+struct AtMisc {
+  int rows[kAtRowCap];  // gather row coordinates
+  float cs[kAtMaxRope / 2], sn[kAtMaxRope / 2];
+  uint64_t full[kAtMaxSlots], empty[kAtMaxSlots];
+  uint64_t s_full[2], p_full[2], pv_done[2], q_tma, q_ready, rows_ready, rope_ready;
+  uint32_t tmem_base;
+  int n_rows;  // padded rows (multiple of 4)
+  int n_sel;   // selected rows (valid rows [0, n_sel))
+  int n_win;   // window rows (valid rows [pad4(n_sel), pad4(n_sel) + n_win))
+  int abort_flag;
+  int scan_tmp[4];
+};
+
+template <int NQ>
+struct AtLayout {
+  static constexpr int kSlots = NQ == 2 ? 9 : 13;
+  static constexpr int kOwnChunks = 4 / NQ;         // 128-dim chunks of output dims
+  static constexpr int kOCols = kAtDim / NQ;        // output dims (and O columns)
+  static constexpr int kQOwnSub = NQ == 2 ? 4 : 0;  // q sub-blocks kept in shared memory
+  static constexpr int kQStage = 8 - kQOwnSub;      // q sub-blocks staged for TMEM
+  static constexpr int kRingOff = kQOwnSub * kAtSubBytes;
+  static constexpr int kMiscOff = kRingOff + kSlots * kAtChunkBytes;
+  static constexpr size_t kBytes = (size_t)kMiscOff + sizeof(AtMisc);
+  static constexpr uint32_t kTmemS = kOCols;         // S0, S1: 2 x 64 columns
+  static constexpr uint32_t kTmemQ = kOCols + 128;   // Q chunks held in TMEM
+};
+static_assert(AtLayout<2>::kBytes + 1024 <= 232448, "shared memory budget (NQ = 2)");
+static_assert(AtLayout<4>::kBytes + 1024 <= 232448, "shared memory budget (NQ = 4)");
+
+// 2^x by the hardware approximation (relative error ~2^-22; the softmax
+// weights are rounded to bf16 right after).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -90,13 +122,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "r"(valid ? 16 : 0)
                : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 // Arrive (without changing the expected count) on `bar` once every cp.async
 // this thread issued so far has landed.
@@ -118,33 +143,59 @@ __device__ __forceinline__ uint32_t swz(int r, int u) {
   return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4));
 }
 
-template <bool kHca>
+// cos / sin of pos * freq: the angle is reduced modulo 2 pi in double
+// precision (2 pi split in two parts), then taken in fp32.
+__device__ __forceinline__ void rope_cs_reduced(long long pos, double freq, float* c, float* s) {
+  const double x = (double)pos * freq;
+  const double k = rint(x * 0.15915494309189535);
+  double r = fma(-k, 6.283185307179586, x);
+  r = fma(-k, 2.4492935982947064e-16, r);
+  sincosf((float)r, s, c);
+}
+
+template <bool kHca, int NQ>
 __global__ void __launch_bounds__(kAtThreads, 1)
     k_attn_tc(AttnTcArgs a, const __grid_constant__ CUtensorMap tm_q) {
   using namespace sm100;
+  using Lay = AtLayout<NQ>;
+  constexpr int kSlots = Lay::kSlots;
+  constexpr int kOwn = Lay::kOwnChunks;
+  constexpr int kOCols = Lay::kOCols;
   extern __shared__ uint8_t smem_raw[];
-  AtSmem& sm = *reinterpret_cast<AtSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                          ~static_cast<uintptr_t>(1023));
-  const int half = blockIdx.x & 1;
-  const int split = blockIdx.x >> 1;
+  uint8_t* base_ptr = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                 ~static_cast<uintptr_t>(1023));
+  uint8_t* q_own = base_ptr;                 // kQOwnSub x [128][128 B]
+  uint8_t* ring = base_ptr + Lay::kRingOff;  // kSlots x 16 KB
+  AtMisc& sm = *reinterpret_cast<AtMisc*>(base_ptr + Lay::kMiscOff);
+
+  const int part = blockIdx.x % NQ;
+  const int split = blockIdx.x / NQ;
   const int row_q = blockIdx.y;  // b * Tq + tq
   const int b = row_q / a.Tq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = a.q_pos[row_q];
   const int rope0 = kAtDim - a.rope_dim;
-  const int own0 = 2 * half;  // own 128-dim chunks: own0, own0 + 1 (dims 256*half ..)
-  const int oth0 = 2 * (1 - half);
-  // staging of the other half of q (4 sub-blocks of [128 heads][64 dims])
-  uint8_t* q_stage = sm.r2[kAtR2 - 4];
+  // 128-dim chunks in streaming order: the others first, then the own ones
+  // (own chunks: dims part * kOCols ..)
+  const int own0 = part * kOwn;
+  int chunk_of[4];
+  {
+    int w = 0;
+    for (int c = 0; c < 4; ++c)
+      if (c < own0 || c >= own0 + kOwn) chunk_of[w++] = c;
+    for (int c = 0; c < kOwn; ++c) chunk_of[w++] = own0 + c;
+  }
+  // q sub-block sb (64 dims) lives in shared memory (own half, NQ = 2) or in
+  // TMEM at column 32 * q_tidx(sb); TMEM-bound sub-blocks are staged in the
+  // last ring slots
+  auto q_in_smem = [&](int sb) { return NQ == 2 && (sb >> 2) == part; };
+  auto q_tidx = [&](int sb) { return NQ == 2 ? (sb & 3) : sb; };
+  uint8_t* q_stage = ring + (kSlots - Lay::kQStage) * kAtChunkBytes;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kAtR1; ++s) {
-      mbar_init(&sm.r1_full[s], 128);
-      mbar_init(&sm.r1_empty[s], 1);
-    }
-    for (int s = 0; s < kAtR2; ++s) {
-      mbar_init(&sm.r2_full[s], 128);
-      mbar_init(&sm.r2_empty[s], 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&sm.full[s], 128);
+      mbar_init(&sm.empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
@@ -154,6 +205,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     mbar_init(&sm.q_tma, 1);
     mbar_init(&sm.q_ready, 128);
     mbar_init(&sm.rows_ready, 128);
+    mbar_init(&sm.rope_ready, 32);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -165,45 +217,50 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t t_o = tmem, t_s = tmem + 256, t_q = tmem + 384;
+  const uint32_t t_o = tmem, t_s = tmem + Lay::kTmemS, t_q = tmem + Lay::kTmemQ;
   volatile int* abortp = &sm.abort_flag;
 
   if (warp == 4 && lane == 0) {
-    // q of this token: 8 boxes of [128 heads][64 dims] (128B swizzle); own
-    // half straight to its place, other half to the staging slots
+    // q of this token: 8 boxes of [128 heads][64 dims], 128B swizzle
     tma_prefetch_desc(&tm_q);
     mbar_arrive_expect_tx(&sm.q_tma, kAtHeads * kAtDim * 2);
     for (int sb = 0; sb < 8; ++sb) {
-      const bool own = (sb >> 2) == half;
-      uint8_t* dst = own ? sm.q_own[sb & 3] : q_stage + (sb & 3) * (kAtHeads * 128);
+      uint8_t* dst = q_in_smem(sb) ? q_own + (sb & 3) * kAtSubBytes
+                                   : q_stage + q_tidx(sb) * kAtSubBytes;
       tma_load_2d(dst, &tm_q, &sm.q_tma, sb * 64, row_q * kAtHeads);
     }
   }
-
-  if (warp < 4) {
-    // ======================= softmax / epilogue warps
-    // ---- RoPE table at the query position
-    if (threadIdx.x < a.rope_dim / 2) {
+  if (warp == 8) {
+    // RoPE table at the query position (this warp only issues MMAs once q is
+    // in place)
+    for (int i = lane; i < a.rope_dim / 2; i += 32) {
       float c, s;
-      rope_cos_sin(t, threadIdx.x, a.rope_dim, a.theta, &c, &s);
-      sm.cs[threadIdx.x] = c;
-      sm.sn[threadIdx.x] = s;
+      rope_cs_reduced(t, a.freq[i], &c, &s);
+      sm.cs[i] = c;
+      sm.sn[i] = s;
     }
-    // ---- row list: selected (or visible) entries, then the window's raw rows
+    mbar_arrive(&sm.rope_ready);
+  }
+
+  if (warp >= 4 && warp < 8) {
+    // ======================= row list (warps 4-7, while warps 0-3 stage q):
+    // gather coordinates of the selected (or visible) entries, then the
+    // window's raw rows, each part padded to a multiple of 4 rows
+    const int tid = threadIdx.x - 128;
+    const int cmp_y0 = b * a.n_max;    // row 0 of this sequence in kv_cmp
+    const int raw_y0 = b * a.raw_max;  // row 0 of this sequence in kv_raw
     int base = 0;
     if (kHca) {
-      const int nv = min(n_visible(t, a.n_cmp[b], a.width, a.stride), a.n_max);
-      for (int j = threadIdx.x; j < nv; j += 128)
-        if (j < kAtRowCap) sm.rows[j] = j;
+      const int nv = min(min(n_visible(t, a.n_cmp[b], a.width, a.stride), a.n_max), kAtRowCap);
+      for (int j = tid; j < nv; j += 128) sm.rows[j] = cmp_y0 + j;
       base = nv;
     } else {
-      __shared__ int scan_tmp[4];
       const int* sel = a.idx + (size_t)row_q * a.topk;
       constexpr int kMaxK = kAtRowCap / 128;
       int jv[kMaxK];
 #pragma unroll
-      for (int k = 0; k < kMaxK; ++k) {  // all loads in flight at once
-        const int i = k * 128 + threadIdx.x;
+      for (int k = 0; k < kMaxK; ++k) {  // every load in flight at once
+        const int i = k * 128 + tid;
         jv[k] = i < a.topk ? sel[i] : -1;
       }
 #pragma unroll
@@ -221,55 +278,72 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const int n = __shfl_up_sync(0xffffffffu, x, o);
           if (lane >= o) x += n;
         }
-        if (lane == 31) scan_tmp[warp] = x;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (lane == 31) sm.scan_tmp[warp - 4] = x;
+        asm volatile("bar.sync 2, 128;" ::: "memory");
         int off = 0, tot = 0;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const int c = scan_tmp[w];
-          off += w < warp ? c : 0;
+          const int c = sm.scan_tmp[w];
+          off += w < warp - 4 ? c : 0;
           tot += c;
         }
-        if (v && base + off + x - 1 < kAtRowCap) sm.rows[base + off + x - 1] = j;
+        if (v && base + off + x - 1 < kAtRowCap) sm.rows[base + off + x - 1] = cmp_y0 + j;
         base += tot;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 2, 128;" ::: "memory");
       }
+      base = min(base, kAtRowCap);
     }
+    const int n_sel = base;
+    const int ps = (n_sel + 3) & ~3;
+    for (int k = n_sel + tid; k < ps; k += 128) sm.rows[k] = cmp_y0;  // masked padding
     {
       const int rp0 = a.raw_pos0[b];
       const int w_lo = max(max(0, t - a.window + 1), rp0);
       const int w_hi = min(t, rp0 + min(a.n_raw[b], a.raw_max) - 1);
-      const int n_win = (a.window > 0 && w_hi >= w_lo) ? w_hi - w_lo + 1 : 0;
-      for (int u = threadIdx.x; u < n_win; u += 128)
-        if (base + u < kAtRowCap) sm.rows[base + u] = a.n_max + (w_lo - rp0) + u;
-      if (threadIdx.x == 0) sm.n_rows = min(base + n_win, kAtRowCap);
+      int n_win = (a.window > 0 && w_hi >= w_lo) ? w_hi - w_lo + 1 : 0;
+      n_win = max(0, min(n_win, kAtRowCap - ps));
+      const int pw = (n_win + 3) & ~3;
+      for (int u = tid; u < pw; u += 128)
+        sm.rows[ps + u] = raw_y0 + (w_lo - rp0) + (u < n_win ? u : 0);
+      if (tid == 0) {
+        sm.n_sel = n_sel;
+        sm.n_win = n_win;
+        sm.n_rows = ps + pw;
+      }
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");  // rope table + rows written
+    asm volatile("bar.sync 2, 128;" ::: "memory");  // rows written
     mbar_arrive(&sm.rows_ready);
   }
 
-  // this split's rows (rows_ready orders the reads after the writes)
-  const bool rows_ok = mbar_wait(&sm.rows_ready, 0, abortp);
-  const int R = rows_ok ? sm.n_rows : 0;
-  const int r_lo = (int)((long long)R * split / a.splits);
-  const int r_hi = (int)((long long)R * (split + 1) / a.splits);
-  const int nrow = r_hi - r_lo;
-  const int ntile = (nrow + kAtTile - 1) / kAtTile;
+  // this split's rows, in groups of 4 (each role waits for rows_ready
+  // before reading the list)
+  bool rows_ok = false;
+  int r_lo = 0, r_hi = 0, nrow = 0, ntile = 0;
+  auto load_split = [&]() {
+    rows_ok = mbar_wait(&sm.rows_ready, 0, abortp);
+    const int G = rows_ok ? sm.n_rows / 4 : 0;
+    r_lo = 4 * (int)((long long)G * split / a.splits);
+    r_hi = 4 * (int)((long long)G * (split + 1) / a.splits);
+    nrow = r_hi - r_lo;
+    ntile = (nrow + kAtTile - 1) / kAtTile;
+  };
 
   if (warp < 4) {
+    // ======================= softmax / epilogue warps
     const int head = warp * 32 + lane;  // TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    // ---- q: other half from staging to TMEM, RoPE on the rotated dims,
-    //      rounded to bf16
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_tma, 0, abortp));
+    // ---- q: staged sub-blocks to TMEM, RoPE on the rotated dims, bf16
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_tma, 0, abortp) &&
+                                              mbar_wait(&sm.rope_ready, 0, abortp));
     if (ok) {
 #pragma unroll 1
-      for (int sbi = 0; sbi < 8; ++sbi) {
-        const bool own = (sbi >> 2) == half;
-        const int d0 = sbi * 64;
+      for (int sb = 0; sb < 8; ++sb) {
+        const bool in_smem = q_in_smem(sb);
+        const int d0 = sb * 64;
         const bool rot = d0 + 64 > rope0;
-        if (own && !rot) continue;
-        uint8_t* blk = own ? sm.q_own[sbi & 3] : q_stage + (sbi & 3) * (kAtHeads * 128);
+        if (in_smem && !rot) continue;
+        uint8_t* blk = in_smem ? q_own + (sb & 3) * kAtSubBytes
+                               : q_stage + q_tidx(sb) * kAtSubBytes;
         uint32_t w[32];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -291,13 +365,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
           }
         }
-        if (own) {
+        if (in_smem) {
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<uint4*>(blk + swz(head, u)) =
                 make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         } else {
-          const uint32_t col = (uint32_t)((sbi & 3) * 32);
+          const uint32_t col = (uint32_t)(q_tidx(sb) * 32);
           uint32_t r16[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) r16[e] = w[e];
@@ -312,8 +386,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     fence_proxy_async();
     tc_fence_before();
     mbar_arrive(&sm.q_ready);
+    load_split();
+    ok = ok && __all_sync(0xffffffffu, rows_ok);
 
     // ---- online softmax over the tiles
+    const int n_sel = sm.n_sel, ps = (n_sel + 3) & ~3, pe = ps + sm.n_win;
     float m_run = -INFINITY, l_run = 0.f;
     for (int i = 0; i < ntile && ok; ++i) {
       const int sb = i & 1;
@@ -321,7 +398,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], ph, abortp));
       if (!ok) break;
       tc_fence_after();
-      const int valid = min(kAtTile, nrow - i * kAtTile);
+      const int g0 = r_lo + i * kAtTile;  // list index of row 0 of the tile
       float z[64];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -334,7 +411,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       float mt = -INFINITY;
 #pragma unroll
       for (int e = 0; e < 64; ++e) {
-        if (e >= valid) z[e] = -INFINITY;
+        const int g = g0 + e;
+        const bool valid = g < r_hi && (g < n_sel || (g >= ps && g < pe));
+        if (!valid) z[e] = -INFINITY;
         mt = fmaxf(mt, z[e]);
       }
       if (mt > m_run + kAtRescaleLog2 || m_run == -INFINITY) {
@@ -346,7 +425,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           tc_fence_after();
           const float alpha = exp2f(m_run - mt);
 #pragma unroll 1
-          for (int cc = 0; cc < 256; cc += 32) {
+          for (int cc = 0; cc < kOCols; cc += 32) {
             uint32_t r[32];
             tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
             tmem_wait_ld();
@@ -367,7 +446,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       float psum = 0.f;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = exp2f(z[2 * e] - m_run), p1 = exp2f(z[2 * e + 1] - m_run);
+        const float p0 = ex2_approx(z[2 * e] - m_run), p1 = ex2_approx(z[2 * e + 1] - m_run);
         __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
         const float2 back = __bfloat1622float2(pb);
         psum += back.x + back.y;
@@ -389,29 +468,51 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (ok && ntile > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(ntile - 1) & 1],
                                              (uint32_t)((ntile - 1) >> 1) & 1u, abortp));
+    // The ring is idle once the last PV has landed: each 32-column slab of O
+    // is staged there ([128 heads][32 + 1 floats], padded against bank
+    // conflicts) and written out as whole 128-byte row segments.
+    float* stage = reinterpret_cast<float*>(ring);
+    constexpr int kStageLd = 33;
+    {  // all four softmax warps agree before the barriers below
+      uint32_t all;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+          "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(all)
+          : "r"(ok ? 1u : 0u)
+          : "memory");
+      ok = all != 0;
+    }
     if (ok) {
       tc_fence_after();
       const float sink_l2 = a.sink[head] * 1.4426950408889634f;
+      float scl = 1.f;
       if (a.splits == 1) {
         const float mm = fmaxf(m_run, sink_l2);
         const float den = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - mm)) +
                           exp2f(sink_l2 - mm);
-        const float scl = (m_run == -INFINITY || !(den > 0.f)) ? 0.f : exp2f(m_run - mm) / den;
-        __nv_bfloat16* dst = a.out + ((size_t)row_q * kAtHeads + head) * kAtDim + half * 256;
+        scl = (m_run == -INFINITY || !(den > 0.f)) ? 0.f : exp2f(m_run - mm) / den;
+      } else {
+        const size_t unit = ((size_t)row_q * a.splits + split) * NQ + part;
+        float* pml = a.part_ml + unit * 2 * kAtHeads;
+        pml[head] = m_run;
+        pml[kAtHeads + head] = l_run;
+      }
 #pragma unroll 1
-        for (int cc = 0; cc < 256; cc += 32) {
-          float o[32];
-          if (ntile > 0) {
-            uint32_t r[32];
-            tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
-            tmem_wait_ld();
+      for (int cc = 0; cc < kOCols; cc += 32) {
+        float o[32];
+        if (ntile > 0) {
+          uint32_t r[32];
+          tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(r[e]) * scl;
-          } else {
+          for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(r[e]) * scl;
+        } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = 0.f;
-          }
-          const int d0 = half * 256 + cc;
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+        if (a.splits == 1) {
+          const int d0 = part * kOCols + cc;
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const int d = d0 + e;
@@ -422,105 +523,80 @@ __global__ void __launch_bounds__(kAtThreads, 1)
               o[e + 1] = -x0 * sm.sn[ii] + x1 * sm.cs[ii];
             }
           }
-          uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            d4[u] = make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]),
-                               pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
-                               pack_bf16x2(o[8 * u + 4], o[8 * u + 5]),
-                               pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
         }
-      } else {
-        const size_t unit = ((size_t)row_q * a.splits + split) * 2 + half;
-        float* po = a.part_o + (unit * kAtHeads + head) * 256;
-#pragma unroll 1
-        for (int cc = 0; cc < 256; cc += 32) {
-          float4* d4 = reinterpret_cast<float4*>(po + cc);
-          if (ntile > 0) {
-            uint32_t r[32];
-            tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
-            tmem_wait_ld();
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // previous slab written out
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              d4[u] = make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                                  __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3]));
-          } else {
+        for (int e = 0; e < 32; ++e) stage[head * kStageLd + e] = o[e];
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (a.splits == 1) {
+          // 128 rows x 64 B (bf16): 4 lanes per row, 16 B each
+          __nv_bfloat16* dst0 = a.out + (size_t)row_q * kAtHeads * kAtDim + part * kOCols + cc;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) d4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int k = 0; k < 4; ++k) {
+            const int rr = k * 32 + (threadIdx.x >> 2), q = threadIdx.x & 3;
+            const float* src = stage + rr * kStageLd + q * 8;
+            *reinterpret_cast<uint4*>(dst0 + (size_t)rr * kAtDim + q * 8) =
+                make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                           pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+          }
+        } else {
+          // 128 rows x 128 B (fp32): 8 lanes per row, 16 B each
+          const size_t unit = ((size_t)row_q * a.splits + split) * NQ + part;
+          float* dst0 = a.part_o + unit * kAtHeads * kOCols + cc;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rr = k * 16 + (threadIdx.x >> 3), q = threadIdx.x & 7;
+            const float* src = stage + rr * kStageLd + q * 4;
+            *reinterpret_cast<float4*>(dst0 + (size_t)rr * kOCols + q * 4) =
+                make_float4(src[0], src[1], src[2], src[3]);
           }
         }
-        float* pml = a.part_ml + unit * 2 * kAtHeads;
-        pml[head] = m_run;
-        pml[kAtHeads + head] = l_run;
       }
     }
   } else if (warp < 8) {
     // ======================= gather producers (128 threads)
+    // Chunk n (tile n / 4, part n % 4 in streaming order) goes to ring slot
+    // n % kSlots.  Every thread waits for the slot itself and issues its own
+    // 8 copies of each chunk (rows (pt >> 4) + 8 m, 16-byte unit pt & 15): no
+    // barrier among the producers, so the copy issue never waits on the
+    // slowest thread.  Rows past the split end are zero-filled (masked).
+    load_split();
     const int pt = threadIdx.x - 128;
-    const __nv_bfloat16* cmp = a.kv_cmp + (size_t)b * a.n_max * kAtDim;
-    const __nv_bfloat16* raw = a.kv_raw + (size_t)b * a.raw_max * kAtDim;
-    int n1 = 0, n2 = 0;  // chunks issued into each ring
+    const int q16 = pt & 15;
+    const int r0 = pt >> 4;
+    const int n_sel = sm.n_sel, ps = (n_sel + 3) & ~3;
     bool okp = rows_ok;
     bool staged = false;  // q staging slots handed back
+    int n = 0;
     for (int i = 0; i < ntile && okp; ++i) {
-      const int tb = i & 1;
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      if (pt < kAtTile) {
-        const int r = r_lo + i * kAtTile + pt;
-        const __nv_bfloat16* p = nullptr;
-        if (r < r_hi) {
-          const int id = sm.rows[r];
-          p = id < a.n_max ? cmp + (size_t)id * kAtDim : raw + (size_t)(id - a.n_max) * kAtDim;
-        }
-        sm.row_ptr[tb][pt] = p;
-      }
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      for (int ck = 0; ck < 4; ++ck) {
-        const bool own = ck >= 2;
-        const int chunk = own ? own0 + (ck - 2) : oth0 + ck;
-        int slot;
-        uint64_t* full;
-        uint8_t* base;
-        // one elected thread waits for the slot; the decision is shared so
-        // that all 128 producers leave the loop together
-        if (!own) {
-          slot = n1 % kAtR1;
-          if (pt == 0)
-            sm.prod_ok = mbar_wait(&sm.r1_empty[slot], ((uint32_t)(n1 / kAtR1) & 1u) ^ 1u, abortp);
-          full = &sm.r1_full[slot];
-          base = sm.r1[slot];
-          ++n1;
-        } else {
-          slot = n2 % kAtR2;
-          if (pt == 0) {
-            bool w = mbar_wait(&sm.r2_empty[slot], ((uint32_t)(n2 / kAtR2) & 1u) ^ 1u, abortp);
-            if (w && !staged && slot >= kAtR2 - 4) {  // slot still holds q staging
-              w = mbar_wait(&sm.q_ready, 0, abortp);
-              staged = true;
-            }
-            sm.prod_ok = w;
-          }
-          full = &sm.r2_full[slot];
-          base = sm.r2[slot];
-          ++n2;
-        }
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-        okp = sm.prod_ok != 0;
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-        if (!okp) break;
-        const uint32_t dst0 = smem_u32(base);
+      const __nv_bfloat16* rp[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int piece = pt + 128 * k;  // 0..1023
-          const int r = piece >> 4;        // row in tile
-          const int q16 = piece & 15;      // 16 B unit within the 256 B chunk
-          const __nv_bfloat16* rp = sm.row_ptr[tb][r];
-          const void* src = rp ? (const void*)(rp + chunk * 128 + q16 * 8) : (const void*)a.q;
-          const uint32_t dst = dst0 + (uint32_t)((q16 >> 3) * (kAtChunkBytes / 2)) +
-                               swz(r, q16 & 7);
-          cp_async16(dst, src, rp != nullptr);
+      for (int m = 0; m < 8; ++m) {
+        const int g = r_lo + i * kAtTile + r0 + 8 * m;
+        rp[m] = nullptr;
+        if (g < r_hi) {
+          const int y = sm.rows[g];
+          rp[m] = (g < ps ? a.kv_cmp : a.kv_raw) + (size_t)y * kAtDim;
         }
-        cp_async_arrive(full);  // completes the chunk's phase when the copies land
+      }
+      for (int ck = 0; ck < 4; ++ck, ++n) {
+        const int chunk = chunk_of[ck];
+        const int slot = n % kSlots;
+        okp = mbar_wait_backoff(&sm.empty[slot], ((uint32_t)(n / kSlots) & 1u) ^ 1u, abortp);
+        if (okp && !staged && slot >= kSlots - Lay::kQStage) {  // slot still holds q staging
+          okp = mbar_wait_backoff(&sm.q_ready, 0, abortp);
+          staged = true;
+        }
+        if (!okp) break;
+        const uint32_t dst0 = smem_u32(ring + slot * kAtChunkBytes) +
+                              (uint32_t)((q16 >> 3) * (kAtChunkBytes / 2));
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int r = r0 + 8 * m;
+          const void* src = rp[m] ? (const void*)(rp[m] + chunk * 128 + q16 * 8) : (const void*)a.q;
+          cp_async16(dst0 + swz(r, q16 & 7), src, rp[m] != nullptr);
+        }
+        cp_async_arrive(&sm.full[slot]);  // completes when the copies land
       }
     }
     cp_async_wait_all();
@@ -528,81 +604,83 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // ======================= MMA issuer
     constexpr uint32_t id_qk = idesc_bf16_f32(128, kAtTile);
     constexpr uint32_t id_pv = idesc_bf16_f32(128, 128, 0, 1);
-    int c1 = 0, c2 = 0;  // chunks consumed per ring
-    int own_slot[2][2];
+    int n = 0;  // chunks consumed
+    int own_slot[2][kOwn];
     int last_pv = -1, last_s = -1;
+    load_split();
     bool okm = rows_ok && mbar_wait(&sm.q_ready, 0, abortp);
     tc_fence_after();
-    const uint32_t qs = smem_u32(sm.q_own[0]);
+    const uint32_t qs = smem_u32(q_own);
     auto issue_pv = [&](int j) -> bool {
       const int sb = j & 1;
       if (!mbar_wait(&sm.p_full[sb], (uint32_t)(j >> 1) & 1u, abortp)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int ks = 0; ks < kAtTile / 16; ++ks) {
+      for (int oc = 0; oc < kOwn; ++oc) {
+        const uint64_t vd0 =
+            sw128_desc(smem_u32(ring + own_slot[sb][oc] * kAtChunkBytes), kAtChunkBytes / 2, 1024);
 #pragma unroll
-        for (int oc = 0; oc < 2; ++oc) {
-          const uint32_t vb = smem_u32(sm.r2[own_slot[sb][oc]]) + (uint32_t)(ks * 16 * 128);
-          const uint64_t bd = sw128_desc(vb, kAtChunkBytes / 2, 1024);
-          mma_ts(t_o + (uint32_t)(oc * 128), t_s + (uint32_t)(sb * 64 + ks * 8), bd, id_pv,
-                 (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kAtTile / 16; ++ks)
+          mma_ts(t_o + (uint32_t)(oc * 128), t_s + (uint32_t)(sb * 64 + ks * 8),
+                 vd0 + (uint64_t)((ks * 16 * 128) >> 4), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
       }
-      tc_commit(&sm.r2_empty[own_slot[sb][0]]);
-      tc_commit(&sm.r2_empty[own_slot[sb][1]]);
+#pragma unroll
+      for (int oc = 0; oc < kOwn; ++oc) tc_commit(&sm.empty[own_slot[sb][oc]]);
       tc_commit(&sm.pv_done[sb]);
       last_pv = j;
       return true;
     };
+    int pv_next = 0;  // next tile whose PV is still to be issued
     for (int i = 0; i < ntile && okm; ++i) {
       const int sb = i & 1;
       if (i >= 2) {  // P(i-2) lives in S[sb]: its PV must have finished
+        if (pv_next <= i - 2) okm = issue_pv(pv_next++);
+        if (!okm) break;
         okm = mbar_wait(&sm.pv_done[sb], (uint32_t)((i - 2) >> 1) & 1u, abortp);
         if (!okm) break;
         tc_fence_after();
       }
-      // S(i) = Q K_i^T over the four 128-dim chunks (other half first)
-      for (int ck = 0; ck < 4 && okm; ++ck) {
-        const bool own = ck >= 2;
-        int slot;
-        if (!own) {
-          slot = c1 % kAtR1;
-          okm = mbar_wait(&sm.r1_full[slot], (uint32_t)(c1 / kAtR1) & 1u, abortp);
-          ++c1;
-        } else {
-          slot = c2 % kAtR2;
-          okm = mbar_wait(&sm.r2_full[slot], (uint32_t)(c2 / kAtR2) & 1u, abortp);
-          own_slot[sb][ck - 2] = slot;
-          ++c2;
-        }
+      // S(i) = Q K_i^T over the four 128-dim chunks (others first)
+      for (int ck = 0; ck < 4 && okm; ++ck, ++n) {
+        const int chunk = chunk_of[ck];
+        const bool own = ck >= 4 - kOwn;
+        const int slot = n % kSlots;
+        okm = mbar_wait(&sm.full[slot], (uint32_t)(n / kSlots) & 1u, abortp);
+        if (own) own_slot[sb][ck - (4 - kOwn)] = slot;
         if (!okm) break;
-        // the chunk was written by cp.async (generic proxy); the MMA reads it
-        // through the async proxy
+        // written by cp.async (generic proxy), read by the MMA (async proxy)
         fence_proxy_async();
         tc_fence_after();
-        const uint32_t kb = smem_u32(own ? sm.r2[slot] : sm.r1[slot]);
+        // descriptors: one per chunk, k steps by adding (offset >> 4) to the
+        // start-address field
+        const uint64_t bd0 = sw128_desc(smem_u32(ring + slot * kAtChunkBytes), 16, 1024);
+        const int sbq0 = chunk * 2;
+        if (!q_in_smem(sbq0)) {
+          const uint32_t a0 = t_q + (uint32_t)(q_tidx(sbq0) * 32);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bd = sw128_desc(kb + (uint32_t)((ks >> 2) * (kAtChunkBytes / 2) +
-                                                         (ks & 3) * 32), 16, 1024);
-          const uint32_t acc = (ck | ks) != 0 ? 1u : 0u;
-          if (!own) {
-            mma_ts(t_s + (uint32_t)(sb * 64), t_q + (uint32_t)(ck * 64 + ks * 8), bd, id_qk, acc);
-          } else {
-            const int sbq = (ck - 2) * 2 + (ks >> 2);
-            const uint64_t ad = sw128_desc(qs + (uint32_t)(sbq * kAtHeads * 128 + (ks & 3) * 32),
-                                           16, 1024);
-            mma_ss(t_s + (uint32_t)(sb * 64), ad, bd, id_qk, acc);
-          }
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ts(t_s + (uint32_t)(sb * 64), a0 + (uint32_t)((ks >> 2) * 32 + (ks & 3) * 8),
+                   bd0 + (uint64_t)(((ks >> 2) * (kAtChunkBytes / 2) + (ks & 3) * 32) >> 4),
+                   id_qk, (ck | ks) != 0 ? 1u : 0u);
+        } else {
+          const uint64_t ad0 = sw128_desc(qs + (uint32_t)((sbq0 & 3) * kAtSubBytes), 16, 1024);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_ss(t_s + (uint32_t)(sb * 64),
+                   ad0 + (uint64_t)(((ks >> 2) * kAtSubBytes + (ks & 3) * 32) >> 4),
+                   bd0 + (uint64_t)(((ks >> 2) * (kAtChunkBytes / 2) + (ks & 3) * 32) >> 4),
+                   id_qk, (ck | ks) != 0 ? 1u : 0u);
         }
-        if (!own) tc_commit(&sm.r1_empty[slot]);
+        if (!own) tc_commit(&sm.empty[slot]);
+        // the previous tile's PV goes in as soon as its P is ready
+        if (pv_next == i - 1 && mbar_try_wait(&sm.p_full[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u))
+          okm = issue_pv(pv_next++);
       }
       if (!okm) break;
       tc_commit(&sm.s_full[sb]);
       last_s = i;
-      if (i >= 1) okm = issue_pv(i - 1);
     }
-    if (okm && ntile > 0) okm = issue_pv(ntile - 1);
+    while (okm && pv_next < ntile) okm = issue_pv(pv_next++);
     // TMEM is freed only after the last MMAs have landed
     int never = 0;
     if (last_s >= 0)
@@ -625,19 +703,23 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
 // Split-KV merge: per (query token, head, dim) the partials (m_s, l_s, O_s)
 // of every split, the sink and the inverse output rotation.  One block per
-// (query token, output half, 8 heads); a thread owns 8 consecutive dims.
+// (query token, output part, 8 heads); a lane owns 512 / NQ / 32 consecutive
+// dims of one head.
+template <int NQ>
 __global__ void __launch_bounds__(256) k_attn_combine(AttnTcArgs a) {
-  __shared__ float cs[256], sn[256];
+  constexpr int kOCols = kAtDim / NQ;
+  constexpr int kPer = kOCols / 32;  // 8 or 4
+  __shared__ float cs[kAtMaxRope / 2], sn[kAtMaxRope / 2];
   const int row_q = blockIdx.x;
-  const int half = blockIdx.y;
+  const int part = blockIdx.y;
   const int head = blockIdx.z * 8 + (threadIdx.x >> 5);
-  const int c0 = (threadIdx.x & 31) * 8;  // dims half*256 + c0 .. + 7
+  const int c0 = (threadIdx.x & 31) * kPer;  // dims part * kOCols + c0 ..
   const int t = a.q_pos[row_q];
   const int rope0 = kAtDim - a.rope_dim;
   const int S = a.splits;
   if (threadIdx.x < a.rope_dim / 2) {
     float c, s;
-    rope_cos_sin(-(long long)t, threadIdx.x, a.rope_dim, a.theta, &c, &s);
+    rope_cs_reduced(t, a.freq[threadIdx.x], &c, &s);
     cs[threadIdx.x] = c;
     sn[threadIdx.x] = s;
   }
@@ -645,41 +727,51 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnTcArgs a) {
   const float sink_l2 = a.sink[head] * 1.4426950408889634f;
   float M = sink_l2;
   for (int s = 0; s < S; ++s) {
-    const size_t unit = ((size_t)row_q * S + s) * 2 + half;
+    const size_t unit = ((size_t)row_q * S + s) * NQ + part;
     M = fmaxf(M, a.part_ml[unit * 2 * kAtHeads + head]);
   }
   float L = exp2f(sink_l2 - M);
-  float o[8];
+  float o[kPer];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) o[e] = 0.f;
+  for (int e = 0; e < kPer; ++e) o[e] = 0.f;
   for (int s = 0; s < S; ++s) {
-    const size_t unit = ((size_t)row_q * S + s) * 2 + half;
+    const size_t unit = ((size_t)row_q * S + s) * NQ + part;
     const float m = a.part_ml[unit * 2 * kAtHeads + head];
     if (m == -INFINITY) continue;
     const float w = exp2f(m - M);
     L += a.part_ml[unit * 2 * kAtHeads + kAtHeads + head] * w;
-    const float4* src = reinterpret_cast<const float4*>(a.part_o + (unit * kAtHeads + head) * 256 + c0);
-    const float4 v0 = src[0], v1 = src[1];
-    o[0] += v0.x * w; o[1] += v0.y * w; o[2] += v0.z * w; o[3] += v0.w * w;
-    o[4] += v1.x * w; o[5] += v1.y * w; o[6] += v1.z * w; o[7] += v1.w * w;
+    const float4* src =
+        reinterpret_cast<const float4*>(a.part_o + (unit * kAtHeads + head) * kOCols + c0);
+#pragma unroll
+    for (int q4 = 0; q4 < kPer / 4; ++q4) {
+      const float4 v = src[q4];
+      o[4 * q4] += v.x * w;
+      o[4 * q4 + 1] += v.y * w;
+      o[4 * q4 + 2] += v.z * w;
+      o[4 * q4 + 3] += v.w * w;
+    }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; e += 2) {
+  for (int e = 0; e < kPer; e += 2) {
     float x0 = o[e] * inv, x1 = o[e + 1] * inv;
-    const int d = half * 256 + c0 + e;
-    if (d >= rope0) {
+    const int d = part * kOCols + c0 + e;
+    if (d >= rope0) {  // inverse rotation at -t
       const float c = cs[(d - rope0) >> 1], s = sn[(d - rope0) >> 1];
-      const float y0 = x0 * c - x1 * s, y1 = x0 * s + x1 * c;
+      const float y0 = x0 * c + x1 * s, y1 = -x0 * s + x1 * c;
       x0 = y0;
       x1 = y1;
     }
     o[e] = x0;
     o[e + 1] = x1;
   }
-  *reinterpret_cast<uint4*>(a.out + ((size_t)row_q * kAtHeads + head) * kAtDim + half * 256 + c0) =
-      make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                 pack_bf16x2(o[6], o[7]));
+  __nv_bfloat16* dst = a.out + ((size_t)row_q * kAtHeads + head) * kAtDim + part * kOCols + c0;
+  if (kPer == 8) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                                pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+  } else {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+  }
 }
 
 }  // namespace csa

@@ -18,6 +18,7 @@
 #include "indexer_simt.cuh"
 #include "indexer_tc.cuh"
 #include "topk.cuh"
+#include "topk_block.cuh"
 
 namespace csa {
 namespace {
@@ -195,22 +196,48 @@ size_t scores_bytes(int B, int Tq, int n_max) {
   return round_up((size_t)B * Tq * (size_t)n_max * sizeof(float), 256);
 }
 
+// Top-k plan: one block per row (candidates in registers) up to 16384
+// entries; two stages (per-chunk top-k, then a merge of the candidates) up to
+// 16 chunks of 16384 when the merge fits one block; else the generic
+// shared-memory radix select.
+constexpr int kTopkChunk = 1024 * 16;
+int topk_chunks(const csa_params_t* p, int n_max) {
+  if (n_max <= kTopkChunk) return 1;
+  const int c = (n_max + kTopkChunk - 1) / kTopkChunk;
+  if (c <= 64 && (long long)c * p->topk <= kTopkChunk) return c;
+  return 0;  // generic path
+}
+
+size_t topk_ws_bytes(const csa_params_t* p, int B, int Tq, int n_max) {
+  const int c = topk_chunks(p, n_max);
+  if (c <= 1) return 0;
+  const size_t rows = (size_t)B * Tq;
+  return round_up(rows * c * (size_t)p->topk * sizeof(int), 256) +
+         round_up(rows * c * sizeof(int), 256);
+}
+
 int num_sms();
 
 // Tensor-core attention applies to the measured head shape in bf16.
 bool attn_tc_ok(const csa_params_t* p, csa_dtype_t dtype, bool hca, int n_max) {
   if (dtype != CSA_BF16 || p->d != kAtDim || p->n_heads != kAtHeads) return false;
-  if (p->rope_dim > kAtDim) return false;
+  if (p->rope_dim > kAtMaxRope) return false;
   const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
-  return rows <= kAtRowCap;
+  return rows + 8 <= kAtRowCap;
 }
 
-// KV splits per query token: enough CTA pairs to cover the SMs, at least one
+// Output-dim parts per query.  Two CTAs per query (q half in TMEM, half in
+// shared memory) measured faster than four (whole q in TMEM, deeper gather
+// ring, four-fold S recompute) on every workload here, so NQ = 4 is kept
+// compiled but not selected.
+int attn_nq(int B, int Tq) { (void)B; (void)Tq; return 2; }
+
+// KV splits per query token: enough CTAs to cover the SMs, at least one
 // 64-row tile per split.
 int attn_splits(const csa_params_t* p, bool hca, int B, int Tq, int n_max) {
-  const long long units = (long long)B * Tq;
+  const long long units = (long long)B * Tq * attn_nq(B, Tq);
   const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
-  long long s = num_sms() / (2 * units);
+  long long s = num_sms() / units;
   const long long max_s = (rows + kAtTile - 1) / kAtTile;
   if (s > max_s) s = max_s;
   if (s > 32) s = 32;
@@ -222,8 +249,8 @@ size_t attn_ws_bytes(const csa_params_t* p, csa_dtype_t dtype, bool hca, int B, 
   if (!attn_tc_ok(p, dtype, hca, n_max)) return 0;
   const int sp = attn_splits(p, hca, B, Tq, n_max);
   if (sp == 1) return 0;
-  const size_t units = (size_t)B * Tq * sp * 2;
-  return round_up(units * kAtHeads * 256 * sizeof(float), 256) +
+  const size_t units = (size_t)B * Tq * sp * attn_nq(B, Tq);
+  return round_up(units * kAtHeads * (kAtDim / attn_nq(B, Tq)) * sizeof(float), 256) +
          round_up(units * 2 * kAtHeads * sizeof(float), 256);
 }
 
@@ -260,8 +287,10 @@ CSA_API csa_status_t csa_workspace_size(const csa_params_t* p, csa_op_t op, int3
   CSA_CHECK(check_sizes(B, Tq, n_max));
   switch (op) {
     case CSA_OP_COMPRESS: *bytes = 0; return CSA_OK;
-    case CSA_OP_TOPK_SELECT: *bytes = 0; return CSA_OK;
-    case CSA_OP_INDEX_TOPK: *bytes = scores_bytes(B, Tq, n_max); return CSA_OK;
+    case CSA_OP_TOPK_SELECT: *bytes = topk_ws_bytes(p, B, Tq, n_max); return CSA_OK;
+    case CSA_OP_INDEX_TOPK:
+      *bytes = scores_bytes(B, Tq, n_max) + topk_ws_bytes(p, B, Tq, n_max);
+      return CSA_OK;
     case CSA_OP_SPARSE_ATTN: *bytes = attn_ws_bytes(p, CSA_BF16, false, B, Tq, n_max); return CSA_OK;
     case CSA_OP_HCA_ATTN: *bytes = attn_ws_bytes(p, CSA_BF16, true, B, Tq, n_max); return CSA_OK;
   }
@@ -360,13 +389,36 @@ static csa_status_t index_scores_impl(const csa_params_t* p, csa_dtype_t dtype, 
 
 static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const int32_t* q_pos,
                               const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
-                              int32_t* idx_out, cudaStream_t s) {
+                              int32_t* idx_out, void* ws, size_t ws_bytes, cudaStream_t s) {
   const unsigned rows = (unsigned)B * (unsigned)Tq;
-  if (n_max >= 8192)
-    k_topk_rows<1024><<<rows, 1024, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, p->topk, p->width,
-                                            p->stride, idx_out);
-  else
-    k_topk_rows<256><<<rows, 256, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, p->topk, p->width,
+  const int k = p->topk;
+  const int chunks = topk_chunks(p, n_max);
+  if (chunks == 1) {
+    if (n_max <= 2048)
+      k_topk_chunk<256, 8><<<dim3(1, rows), 256, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k,
+                                                          p->width, p->stride, 1, idx_out,
+                                                          nullptr, nullptr);
+    else
+      k_topk_chunk<1024, 16><<<dim3(1, rows), 1024, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k,
+                                                            p->width, p->stride, 1, idx_out,
+                                                            nullptr, nullptr);
+    return launched("k_topk_chunk");
+  }
+  if (chunks > 1) {
+    const size_t need = topk_ws_bytes(p, B, Tq, n_max);
+    if (ws_bytes < need)
+      return fail(CSA_ERR_WORKSPACE_TOO_SMALL, "top-k workspace %zu bytes, need %zu", ws_bytes,
+                  need);
+    CSA_CHECK(check_ptr(ws, "ws"));
+    int* cand = (int*)ws;
+    int* cand_n = (int*)((char*)ws + round_up((size_t)rows * chunks * (size_t)k * sizeof(int), 256));
+    k_topk_chunk<1024, 16><<<dim3((unsigned)chunks, rows), 1024, 0, s>>>(
+        scores, q_pos, n_cmp, Tq, n_max, k, p->width, p->stride, chunks, idx_out, cand, cand_n);
+    CSA_CHECK(launched("k_topk_chunk"));
+    k_topk_merge<1024, 16><<<rows, 1024, 0, s>>>(scores, n_max, k, chunks, cand, cand_n, idx_out);
+    return launched("k_topk_merge");
+  }
+  k_topk_rows<1024><<<rows, 1024, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k, p->width,
                                           p->stride, idx_out);
   return launched("k_topk_rows");
 }
@@ -401,9 +453,9 @@ CSA_API csa_status_t csa_topk_select(const csa_params_t* p, const float* scores,
   CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
   CSA_CHECK(check_ptr(idx_out, "idx_out"));
   CSA_CHECK(check_ptr(ws, "ws", true));
-  (void)ws_bytes;
   CSA_CHECK(check_device());
-  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, (cudaStream_t)stream);
+  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, ws, ws_bytes,
+                   (cudaStream_t)stream);
 }
 
 CSA_API csa_status_t csa_index_topk(const csa_params_t* p, csa_dtype_t dtype, const void* q_idx,
@@ -421,7 +473,8 @@ CSA_API csa_status_t csa_index_topk(const csa_params_t* p, csa_dtype_t dtype, co
   CSA_CHECK(check_ptr(q_pos, "q_pos"));
   CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
   CSA_CHECK(check_ptr(idx_out, "idx_out"));
-  const size_t need = scores_bytes(B, Tq, n_max);
+  const size_t sb = scores_bytes(B, Tq, n_max);
+  const size_t need = sb + topk_ws_bytes(p, B, Tq, n_max);
   if (need > 0) CSA_CHECK(check_ptr(ws, "ws"));
   if (ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes, need %zu", ws_bytes, need);
@@ -429,7 +482,8 @@ CSA_API csa_status_t csa_index_topk(const csa_params_t* p, csa_dtype_t dtype, co
   cudaStream_t s = (cudaStream_t)stream;
   float* scores = (float*)ws;
   CSA_CHECK(index_scores_impl(p, dtype, q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, scores, s));
-  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, s);
+  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, (char*)ws + sb, ws_bytes - sb,
+                   s);
 }
 
 static csa_status_t attn_common_checks(const csa_params_t* p, csa_dtype_t dtype, const void* q,
@@ -474,6 +528,27 @@ static csa_status_t launch_attn_simt(const AttnArgs& a, csa_dtype_t dtype, cudaS
   return launched("k_attn_simt");
 }
 
+template <bool kHca, int NQ>
+static csa_status_t launch_attn_tc_nq(const AttnArgs& g, AttnTcArgs& a, int sp, void* ws,
+                                      const CUtensorMap& tq, cudaStream_t s) {
+  using Lay = AtLayout<NQ>;
+  if (sp > 1) {
+    const size_t units = (size_t)g.B * g.Tq * sp * NQ;
+    a.part_o = (float*)ws;
+    a.part_ml = (float*)((char*)ws + round_up(units * kAtHeads * (kAtDim / NQ) * sizeof(float), 256));
+  }
+  const size_t smem = Lay::kBytes + 1024;
+  CSA_CHECK(set_smem_attr(k_attn_tc<kHca, NQ>, smem, "k_attn_tc"));
+  dim3 grid((unsigned)(NQ * sp), (unsigned)(g.B * g.Tq));
+  k_attn_tc<kHca, NQ><<<grid, kAtThreads, smem, s>>>(a, tq);
+  CSA_CHECK(launched("k_attn_tc"));
+  if (sp > 1) {
+    k_attn_combine<NQ><<<dim3((unsigned)(g.B * g.Tq), NQ, kAtHeads / 8), 256, 0, s>>>(a);
+    CSA_CHECK(launched("k_attn_combine"));
+  }
+  return CSA_OK;
+}
+
 template <bool kHca>
 static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, void* ws,
                                    size_t ws_bytes, cudaStream_t s) {
@@ -501,28 +576,16 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   a.stride = g.stride;
   a.rope_dim = g.rope_dim;
   a.scale_log2 = g.scale * 1.4426950408889634f;
-  a.theta = g.theta;
   a.splits = sp;
   a.out = (__nv_bfloat16*)g.out;
   a.part_o = nullptr;
   a.part_ml = nullptr;
-  if (sp > 1) {
-    const size_t units = (size_t)g.B * g.Tq * sp * 2;
-    a.part_o = (float*)ws;
-    a.part_ml = (float*)((char*)ws + round_up(units * kAtHeads * 256 * sizeof(float), 256));
-  }
+  for (int i = 0; i < kAtMaxRope / 2; ++i)
+    a.freq[i] = i < g.rope_dim / 2 ? std::pow(g.theta, -2.0 * i / (double)g.rope_dim) : 0.0;
   CUtensorMap tq;
   CSA_CHECK(make_tmap_bf16(&tq, g.q, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
-  const size_t smem = sizeof(AtSmem) + 1024;
-  CSA_CHECK(set_smem_attr(k_attn_tc<kHca>, smem, "k_attn_tc"));
-  dim3 grid((unsigned)(2 * sp), (unsigned)(g.B * g.Tq));
-  k_attn_tc<kHca><<<grid, kAtThreads, smem, s>>>(a, tq);
-  CSA_CHECK(launched("k_attn_tc"));
-  if (sp > 1) {
-    k_attn_combine<<<dim3((unsigned)(g.B * g.Tq), 2, kAtHeads / 8), 256, 0, s>>>(a);
-    CSA_CHECK(launched("k_attn_combine"));
-  }
-  return CSA_OK;
+  if (attn_nq(g.B, g.Tq) == 4) return launch_attn_tc_nq<kHca, 4>(g, a, sp, ws, tq, s);
+  return launch_attn_tc_nq<kHca, 2>(g, a, sp, ws, tq, s);
 }
 
 static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32_t* q_pos,
@@ -620,18 +683,21 @@ CSA_API csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t d
   CSA_CHECK(check_ptr(q_pos, "q_pos"));
   CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
   CSA_CHECK(check_ptr(idx_out, "idx_out"));
-  const size_t need = (size_t)B * (size_t)Tq * (size_t)n_max;
-  if (need > kNoAllocScoreFloats)
+  // scores first, then the top-k candidate lists of long rows
+  const size_t sb = scores_bytes(B, Tq, n_max);
+  const size_t tb = topk_ws_bytes(p, B, Tq, n_max);
+  if (sb + tb > kNoAllocScoreFloats * sizeof(float))
     return fail(CSA_ERR_UNSUPPORTED_SHAPE,
                 "B*Tq*n_max = %zu scores exceed the no-alloc scratch of %zu; use csa_index_topk "
                 "with a workspace",
-                need, kNoAllocScoreFloats);
+                (size_t)B * (size_t)Tq * (size_t)n_max, kNoAllocScoreFloats);
   CSA_CHECK(check_device());
   float* scores = nullptr;
   CSA_CHECK(noalloc_scores_ptr(&scores));
   cudaStream_t s = (cudaStream_t)stream;
   CSA_CHECK(index_scores_impl(p, dtype, q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, scores, s));
-  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, s);
+  return topk_impl(p, scores, q_pos, n_cmp, B, Tq, n_max, idx_out, (char*)scores + sb,
+                   kNoAllocScoreFloats * sizeof(float) - sb, s);
 }
 
 CSA_API csa_status_t csa_poll_device_error(void* stream) {

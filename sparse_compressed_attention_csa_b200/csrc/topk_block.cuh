@@ -1,0 +1,233 @@
+// Step 2b, fast path: exact top-k ("keeps the top 1,024 entries") of one
+// query row held in registers, ties to the lower index, output ascending.
+//
+// Each of NT threads owns PT consecutive candidates (so thread order then
+// register order is index order).  Radix select on order-preserving uint32
+// keys, 8 bits per pass, starting at the highest bit in which the row's keys
+// differ.  After the last pass the threshold key T and the number of keys
+// equal to T to keep are exact; one pair of block-wide scans over per-thread
+// counts then places every kept index.
+//
+// Rows longer than one block's capacity use two stages: each chunk keeps its
+// own top-k (k_topk_chunk), then the candidates of all chunks, in index
+// order, are selected again (k_topk_merge).  This is exact: an entry in the
+// row's top-k is beaten (higher score, or equal score at a lower index) by
+// fewer than k entries of the row, hence of its chunk.
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+struct TopkShared {
+  unsigned hist[256];
+  int scan[33];
+  uint32_t prefix;
+  int remaining;
+  uint32_t red_and[32], red_or[32];
+};
+
+// Exclusive block scan of one int per thread (also returns the total).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total) {
+  return block_inclusive_scan(v, tmp, total) - v;
+}
+
+// Selects the top `k` of the block's candidates.  key[e], valid[e] describe
+// candidate thread*PT + e; index_of(e) gives its output index.  Writes the
+// kept indices, ascending, to out[0 .. min(k, n_valid)) and returns that
+// count (same value in every thread).
+//
+// The radix passes start at the highest bit in which the valid keys differ
+// (a block AND/OR reduction finds it), so the first digit already spreads
+// over many bins; digits are 8 bits wide from there down to bit 0.  Each
+// pass picks its digit with a 256-thread suffix scan over the histogram.
+template <int NT, int PT, typename IndexOf>
+__device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], int k,
+                          IndexOf index_of, int* out, TopkShared& sh) {
+  static_assert(NT >= 256, "bin scan needs 256 threads");
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int nv_local = 0;
+  uint32_t k_and = 0xffffffffu, k_or = 0u;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    if (valid[e]) {
+      ++nv_local;
+      k_and &= key[e];
+      k_or |= key[e];
+    }
+  }
+  int n_valid;
+  const int before = block_exclusive_scan(nv_local, sh.scan, &n_valid);
+  if (n_valid <= k) {  // keep every valid candidate
+    int p = before;
+#pragma unroll
+    for (int e = 0; e < PT; ++e)
+      if (valid[e]) out[p++] = index_of(e);
+    return n_valid;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    k_and &= __shfl_xor_sync(0xffffffffu, k_and, o);
+    k_or |= __shfl_xor_sync(0xffffffffu, k_or, o);
+  }
+  if (lane == 0) {
+    sh.red_and[wid] = k_and;
+    sh.red_or[wid] = k_or;
+  }
+  __syncthreads();
+  k_and = 0xffffffffu;
+  k_or = 0u;
+  for (int w = 0; w < NT / 32; ++w) {
+    k_and &= sh.red_and[w];
+    k_or |= sh.red_or[w];
+  }
+  const uint32_t diff = k_and ^ k_or;
+  uint32_t prefix, mask;
+  int remaining = k;
+  if (diff == 0u) {  // all valid keys equal
+    prefix = k_and;
+  } else {
+    int hi = 31 - __clz(diff);
+    mask = hi == 31 ? 0u : (0xffffffffu << (hi + 1));  // bits above hi are common
+    prefix = k_and & mask;
+#pragma unroll 1
+    while (hi >= 0) {
+      const int lo = max(hi - 7, 0);
+      const uint32_t dmask = ((hi - lo == 31) ? 0xffffffffu : ((1u << (hi - lo + 1)) - 1u));
+      for (int i = threadIdx.x; i < 256; i += NT) sh.hist[i] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < PT; ++e)
+        if (valid[e] && (key[e] & mask) == prefix)
+          atomicAdd(&sh.hist[(key[e] >> lo) & dmask], 1u);
+      __syncthreads();
+      if (threadIdx.x < 256) {
+        // thread b holds bin 255 - b: an inclusive scan gives, per bin, the
+        // count of keys in this bin or above
+        const int bin = 255 - (int)threadIdx.x;
+        const int h = (int)sh.hist[bin];
+        int x = h;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += n;
+        }
+        if (lane == 31) sh.scan[wid] = x;
+        asm volatile("bar.sync 3, 256;" ::: "memory");
+        int off = 0;
+        for (int w = 0; w < wid; ++w) off += sh.scan[w];
+        const int incl = off + x, excl = incl - h;
+        if (incl >= remaining && excl < remaining) {
+          sh.prefix = prefix | ((uint32_t)bin << lo);
+          sh.remaining = remaining - excl;
+        }
+      }
+      __syncthreads();
+      prefix = sh.prefix;
+      remaining = sh.remaining;
+      mask |= dmask << lo;
+      hi = lo - 1;
+    }
+  }
+  const uint32_t thr = prefix;
+  const int take_eq = remaining;
+  int gt = 0, eq = 0;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    gt += (valid[e] && key[e] > thr) ? 1 : 0;
+    eq += (valid[e] && key[e] == thr) ? 1 : 0;
+  }
+  int eq_tot;
+  const int eq_before = block_exclusive_scan(eq, sh.scan, &eq_tot);
+  const int my_eq = max(0, min(eq, take_eq - eq_before));
+  int sel_tot;
+  int pos = block_exclusive_scan(gt + my_eq, sh.scan, &sel_tot);
+  int eq_taken = 0;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    if (!valid[e]) continue;
+    bool take = key[e] > thr;
+    if (!take && key[e] == thr && eq_taken < my_eq) {
+      take = true;
+      ++eq_taken;
+    }
+    if (take && pos < k) out[pos++] = index_of(e);
+  }
+  return k;
+}
+
+// One CTA per (chunk, query row).  Chunk c covers entries
+// [c * NT * PT, (c + 1) * NT * PT) of the row's visible entries.  With one
+// chunk per row the result goes to idx_out (padded with -1); otherwise to the
+// candidate workspace cand[row][c][k] with its count in cand_n[row][c].
+template <int NT, int PT>
+__global__ void __launch_bounds__(NT)
+    k_topk_chunk(const float* __restrict__ scores, const int* __restrict__ q_pos,
+                 const int* __restrict__ n_cmp, int Tq, int n_max, int k, int width, int stride,
+                 int n_chunks, int* __restrict__ idx_out, int* __restrict__ cand,
+                 int* __restrict__ cand_n) {
+  __shared__ TopkShared sh;
+  const int c = blockIdx.x, row = blockIdx.y;
+  const int b = row / Tq;
+  const int nv = min(n_visible(q_pos[row], n_cmp[b], width, stride), n_max);
+  const int base = c * NT * PT;
+  const float* s = scores + (size_t)row * n_max;
+  uint32_t key[PT];
+  bool valid[PT];
+  const int first = base + threadIdx.x * PT;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    const int j = first + e;
+    valid[e] = j < nv;
+    key[e] = valid[e] ? float_key(s[j]) : 0u;
+  }
+  int* out = n_chunks == 1 ? idx_out + (size_t)row * k : cand + ((size_t)row * n_chunks + c) * k;
+  const int cnt = block_topk<NT, PT>(key, valid, k, [&](int e) { return first + e; }, out, sh);
+  if (n_chunks == 1) {
+    for (int i = cnt + threadIdx.x; i < k; i += NT) out[i] = -1;
+  } else if (threadIdx.x == 0) {
+    cand_n[(size_t)row * n_chunks + c] = cnt;
+  }
+}
+
+// One CTA per query row: the top-k of the concatenated chunk candidates.
+template <int NT, int PT>
+__global__ void __launch_bounds__(NT)
+    k_topk_merge(const float* __restrict__ scores, int n_max, int k, int n_chunks,
+                 const int* __restrict__ cand, const int* __restrict__ cand_n,
+                 int* __restrict__ idx_out) {
+  __shared__ TopkShared sh;
+  __shared__ int offs[65];
+  const int row = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+      offs[c] = acc;
+      acc += cand_n[(size_t)row * n_chunks + c];
+    }
+    offs[n_chunks] = acc;
+  }
+  __syncthreads();
+  const int total = offs[n_chunks];
+  const float* s = scores + (size_t)row * n_max;
+  uint32_t key[PT];
+  bool valid[PT];
+  int idx[PT];
+  const int first = threadIdx.x * PT;
+  int c = 0;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    const int p = first + e;
+    valid[e] = p < total;
+    idx[e] = -1;
+    if (valid[e]) {
+      while (c + 1 < n_chunks && offs[c + 1] <= p) ++c;
+      idx[e] = cand[((size_t)row * n_chunks + c) * k + (p - offs[c])];
+    }
+    key[e] = valid[e] ? float_key(s[idx[e]]) : 0u;
+  }
+  int* out = idx_out + (size_t)row * k;
+  const int cnt = block_topk<NT, PT>(key, valid, k, [&](int e) { return idx[e]; }, out, sh);
+  for (int i = cnt + threadIdx.x; i < k; i += NT) out[i] = -1;
+}
+
+}  // namespace csa
