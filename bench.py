@@ -9,9 +9,10 @@ One step = the whole decode hot path over one batch (32 sequences x 1 query
 token x 128 heads) with the caches resident in HBM.  Each rank runs an
 independent replica of the workload (replicas only: the decode batch
 shards with no exchange), so `scaling` is weak and `value` sums all ranks'
-query-heads over the slowest rank's time.  L2 is flushed (a 256 MiB write)
-before every timed step; each step is a captured CUDA graph whose per-kernel
-durations come from CUDA events recorded inside it.
+query-heads over the slowest rank's time.  L2 is flushed before every timed
+step (a 256 MiB write, then a 256 MiB read, so that no dirty line of the
+flush is left for the step to write back); each step is a captured CUDA graph
+whose per-kernel durations come from CUDA events recorded inside it.
 
 `--impl reference` times the fp64 CPU oracle (the only other place this file
 runs it) on the host cores, one sequence per step.
@@ -20,10 +21,8 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -35,6 +34,33 @@ METRIC = "CSA decode query-heads/s at 64K ctx bs32; % of HBM / bf16 tensor roofl
 UNIT = "query-heads/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_csa_decode_bs32_ctx65536.json")
+
+
+def _source_digest():
+    """Digest of the kernel sources: recorded DRAM traffic is only reported
+    for the kernels it was captured from."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_compressed_attention_csa_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _recorded_traffic(wl):
+    """DRAM bytes per launch group (dram__bytes_read.sum + dram__bytes_write.sum
+    from one ncu capture of this workload), or {} if the kernels changed."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+    except (OSError, ValueError):
+        return {}
+    if rec.get("source_digest") != _source_digest() or rec.get("workload") != wl.name:
+        return {}
+    return {k: v for k, v in rec.get("bytes_per_launch", {}).items()}
 
 
 def _args():
@@ -59,78 +85,95 @@ def _config(wl, extra=None):
     c = {"workload": wl.name, "batch": wl.B, "context": wl.T, "n_cmp": wl.n_cmp,
          "query_heads": wl.n_heads, "head_dim": wl.d, "rope_dim": wl.rope_dim,
          "indexer": f"{wl.idx_heads}x{wl.idx_dim}", "topk": wl.topk, "window": wl.window,
-         "l2": "flushed (256 MiB write) before every timed step", "parallelism": "replicas"}
+         "l2": "flushed before every timed step: 256 MiB write, then 256 MiB read (L2 left clean)",
+         "parallelism": "replicas"}
     if extra:
         c.update(extra)
     return c
 
 
-def algorithmic_bytes(wl):
-    """Bytes one decode step must move at least (caches resident)."""
+def algorithmic_work(wl):
+    """Bytes (and FLOPs) one decode step must move (do) at least, per kernel
+    group and for the whole step, with the caches resident in HBM."""
     B, N, H, d = wl.B, wl.n_cmp, wl.n_heads, wl.d
     keys = B * N * wl.idx_dim * 2
     idx_q = B * wl.idx_heads * wl.idx_dim * 2 + B * wl.idx_heads * 4
-    rows = B * (min(wl.topk, N) + wl.window) * d * 2
+    scores = B * N * 4
+    sel = B * wl.topk * 4
+    n_rows = min(wl.topk, N) + wl.window
+    rows = B * n_rows * d * 2
     q = B * H * d * 2
     out = B * H * d * 2
-    small = B * wl.topk * 4 + H * 4
-    return {"index_scores": keys + idx_q + B * N * 4, "step": keys + idx_q + rows + q + out + small}
+    return {
+        "index_scores": {"bytes": keys + idx_q + scores, "flops": 2 * B * N * wl.idx_heads * wl.idx_dim},
+        "topk_select": {"bytes": scores + sel, "flops": 0},
+        "sparse_attn": {"bytes": rows + q + out + sel + H * 4, "flops": 4 * B * H * n_rows * d},
+        "step": {"bytes": keys + idx_q + rows + q + out + sel + H * 4},
+    }
 
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, max clock and clock-event reasons through NVML every
+    20 ms on a thread, between start() and stop()."""
+    PERIOD_S = 0.02
 
-    def __init__(self, index: int):
-        self.index = index
-        self.lines: list[str] = []
-        self.proc = None
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.rows = []
+        self.stop_evt = threading.Event()
         self.t = None
+        self.handle = None
+        self.nv = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            import torch
+            pr = torch.cuda.get_device_properties(self.dev)
+            try:
+                bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+                self.handle = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.handle = nv.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+        except Exception:
+            self.handle = None
             return
-        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t = threading.Thread(target=self._run, daemon=True)
         self.t.start()
-        deadline = time.time() + 5
-        while not self.lines and time.time() < deadline:
-            time.sleep(0.02)
-        self.mark = len(self.lines)
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return int(fn(self.handle))
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                self.rows.append((nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM),
+                                  nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM),
+                                  self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        end = len(self.lines)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = [l.split(", ") for l in self.lines[self.mark:end] if l]
-        sm = [float(r[1]) for r in rows if len(r) > 8 and r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if len(r) > 8 and r[2].replace(".", "").isdigit()]
-        reasons = set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for r in rows:
-            if len(r) > 8:
-                for n, v in zip(names, r[5:9]):
-                    if v.strip().lower() == "active":
-                        reasons.add(n)
+        if self.t is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable"}
+        self.stop_evt.set()
+        self.t.join(timeout=2)
+        bits = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+        reasons = sorted({n for _, _, r in self.rows for n, b in bits.items() if r & b})
+        sm = [c for c, _, _ in self.rows]
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "sm_max_mhz": max(m for _, m, _ in self.rows) if self.rows else None,
+                "reasons": reasons, "samples": len(sm), "source": "nvml, 20 ms"}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -255,6 +298,11 @@ def run_cuda(args, rank, world, local):
     ws_attn = L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, Bsz, Tq, N)
     ws = torch.empty(max(ws_topk, ws_attn, 256), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)  # 256 MiB
+
+    def flush_l2():
+        flush.zero_()
+        flush_rd.sum()  # evicts the dirty lines of the write: L2 left clean
     stream = torch.cuda.Stream(device=dev)
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
 
@@ -268,9 +316,10 @@ def run_cuda(args, rank, world, local):
                           t["n_raw"], t["sink"], out, ws)
         ev[3].record()
 
-    kernels_per_step = 3
     with torch.cuda.stream(stream):
+        n0 = L.csa_launch_count()
         launch()  # eager warm-up (module load, attribute setup)
+        kernels_per_step = L.csa_launch_count() - n0
     torch.cuda.synchronize()
     L.csa_poll_device_error(stream)
     graph = torch.cuda.CUDAGraph()
@@ -282,7 +331,7 @@ def run_cuda(args, rank, world, local):
         tot = [0.0, 0.0, 0.0, 0.0]
         for _ in range(n):
             with torch.cuda.stream(stream):
-                flush.zero_()
+                flush_l2()
                 graph.replay()
             stream.synchronize()
             a, b, c = (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
@@ -294,7 +343,7 @@ def run_cuda(args, rank, world, local):
         return tot
 
     timed_steps(args.warmup)
-    sampler = ClockSampler(local) if not args.no_clocks else None
+    sampler = ClockSampler(dev) if not args.no_clocks else None
     if sampler:
         sampler.start()
     if world > 1:
@@ -329,7 +378,7 @@ def run_cuda(args, rank, world, local):
 
     def e2e_step():
         with torch.cuda.stream(stream):
-            flush.zero_()
+            flush_l2()
             e_start.record()
             for k in h_in:
                 d_in[k].copy_(h_in[k], non_blocking=True)
@@ -358,25 +407,44 @@ def run_cuda(args, rank, world, local):
         peaks = {}
         if os.path.exists(PEAKS_FILE):
             peaks = json.load(open(PEAKS_FILE))
+        src = "measured" if peaks else "fallback"
         hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-        ab = algorithmic_bytes(wl)
-        t_scores = tot[1] / args.steps * 1e-3
-        achieved = ab["index_scores"] / t_scores / 1e9
+        tc = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        work = algorithmic_work(wl)
+        kernel_ms = {"index_scores": tot[1] / args.steps, "topk_select": tot[2] / args.steps,
+                     "sparse_attn": tot[3] / args.steps}
+        traffic = _recorded_traffic(wl)
+        rl = {}
+        for k, ms in kernel_ms.items():
+            b, f = work[k]["bytes"], work[k]["flops"]
+            gbs = b / (ms * 1e-3) / 1e9
+            tfl = f / (ms * 1e-3) / 1e12
+            # the bound is the roof the kernel's arithmetic intensity meets first
+            tensor = f > 0 and f / b > tc * 1e12 / (hbm * 1e9)
+            rl[k] = {"bound": "tensor" if tensor else "hbm",
+                     "achieved": tfl if tensor else gbs, "peak": tc if tensor else hbm,
+                     "unit": "TFLOP/s" if tensor else "GB/s",
+                     "frac": (tfl / tc) if tensor else (gbs / hbm),
+                     "algorithmic_bytes": b, "flops": f, "ms": ms,
+                     "tensor_frac": tfl / tc if f else 0.0,
+                     "traffic": traffic.get(k), "peak_source": src + " burst"}
+        dom = max(kernel_ms, key=kernel_ms.get)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": _config(wl),
             "gpu_launches": kernels_per_step * args.steps,
-            "kernel_ms": {"index_scores": tot[1] / args.steps, "topk_select": tot[2] / args.steps,
-                          "sparse_attn": tot[3] / args.steps},
-            "step_hbm": {"algorithmic_bytes": ab["step"],
-                         "achieved_gbs": ab["step"] / (step_ms_max * 1e-3) / 1e9,
-                         "frac_of_measured": ab["step"] / (step_ms_max * 1e-3) / 1e9 / hbm},
-            "roofline": {"kernel": "index_scores", "bound": "hbm", "achieved": achieved,
-                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "peak_source": "measured" if peaks else "fallback",
-                         "traffic": None},
+            "kernels_per_step": kernels_per_step,
+            "kernel_ms": kernel_ms,
+            "step_hbm": {"algorithmic_bytes": work["step"]["bytes"],
+                         "achieved_gbs": work["step"]["bytes"] / (step_ms_max * 1e-3) / 1e9,
+                         "frac": work["step"]["bytes"] / (step_ms_max * 1e-3) / 1e9 / hbm,
+                         "peak_source": src},
+            "roofline": dict(kernel=dom, **{k: v for k, v in rl[dom].items()
+                                            if k in ("bound", "achieved", "peak", "unit", "frac",
+                                                     "traffic", "peak_source")}),
+            "roofline_by_kernel": rl,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clocks,

@@ -217,6 +217,11 @@ csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t dtype, co
                                     const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
                                     int32_t* idx_out, void* stream);
 
+/* Number of kernels this library has launched (or recorded into a stream
+ * capture) in this process so far, on every device and host thread.  A
+ * diagnostic: the difference across one call is that call's kernel count. */
+uint64_t csa_launch_count(void);
+
 /* Synchronizes `stream`, then reads and clears the current device's error
  * word: CSA_OK, CSA_ERR_DEVICE_TIMEOUT or CSA_ERR_DEVICE_BOUNDS. */
 csa_status_t csa_poll_device_error(void* stream);

@@ -96,6 +96,8 @@ def _load():
     lib.csa_index_topk_noalloc.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _P, _I, _I, _I, _P,
                                            _P]
     lib.csa_poll_device_error.argtypes = [_P]
+    lib.csa_launch_count.restype = ctypes.c_uint64
+    lib.csa_launch_count.argtypes = []
     for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
               "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error",
               "csa_index_topk_noalloc"):
@@ -263,6 +265,11 @@ def hca_attn(p: Params, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, 
     _req(n_cmp, "n_cmp", torch.int32, 1)
     _attn(_load().hca_attn, p, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, out, ws,
           stream)
+
+
+def csa_launch_count() -> int:
+    """Kernels launched (or captured) by the library so far in this process."""
+    return int(_load().csa_launch_count())
 
 
 def csa_poll_device_error(stream=None):

@@ -52,6 +52,7 @@ constexpr int kAtSubBytes = kAtHeads * 128;       // q box: [128 heads][64 dims]
 constexpr int kAtRowCap = 2048;                   // rows per query token
 constexpr int kAtMaxRope = 128;                   // rotated dims supported
 constexpr int kAtMaxSlots = 13;
+constexpr int kAtMaxSplits = 16;                  // split-KV parts per query token
 constexpr int kAtThreads = 288;
 constexpr float kAtRescaleLog2 = 8.0f;
 
@@ -71,8 +72,9 @@ struct AttnTcArgs {
   float scale_log2;
   int splits;
   __nv_bfloat16* out;  // splits == 1
-  float* part_o;       // splits > 1: [B*Tq][splits][NQ][128][512/NQ]
+  float* part_o;       // splits > 1: [B*Tq][splits][NQ][512/NQ/32][8][128][4]
   float* part_ml;      // [B*Tq][splits][NQ][2][128]  (m, l)
+  int* arrive;         // [B*Tq][NQ] split arrivals, zero before the launch
   double freq[kAtMaxRope / 2];  // RoPE frequencies theta^(-2i/rope_dim)
 };
 
@@ -80,7 +82,7 @@ struct AtMisc {
   int rows[kAtRowCap];  // gather row coordinates
   float cs[kAtMaxRope / 2], sn[kAtMaxRope / 2];
   uint64_t full[kAtMaxSlots], empty[kAtMaxSlots];
-  uint64_t s_full[2], p_full[2], pv_done[2], q_tma, q_ready, rows_ready, rope_ready;
+  uint64_t s_full[2], p_full[2], pv_done[2], q_tma, q_ready, rows_ready, rope_ready, merge_bar;
   uint32_t tmem_base;
   int n_rows;  // padded rows (multiple of 4)
   int n_sel;   // selected rows (valid rows [0, n_sel))
@@ -155,7 +157,8 @@ __device__ __forceinline__ void rope_cs_reduced(long long pos, double freq, floa
 
 template <bool kHca, int NQ>
 __global__ void __launch_bounds__(kAtThreads, 1)
-    k_attn_tc(AttnTcArgs a, const __grid_constant__ CUtensorMap tm_q) {
+    k_attn_tc(AttnTcArgs a, const __grid_constant__ CUtensorMap tm_q,
+              const __grid_constant__ CUtensorMap tm_out) {
   using namespace sm100;
   using Lay = AtLayout<NQ>;
   constexpr int kSlots = Lay::kSlots;
@@ -206,6 +209,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     mbar_init(&sm.q_ready, 128);
     mbar_init(&sm.rows_ready, 128);
     mbar_init(&sm.rope_ready, 32);
+    mbar_init(&sm.merge_bar, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -223,6 +227,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (warp == 4 && lane == 0) {
     // q of this token: 8 boxes of [128 heads][64 dims], 128B swizzle
     tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_out);
     mbar_arrive_expect_tx(&sm.q_tma, kAtHeads * kAtDim * 2);
     for (int sb = 0; sb < 8; ++sb) {
       uint8_t* dst = q_in_smem(sb) ? q_own + (sb & 3) * kAtSubBytes
@@ -468,12 +473,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     if (ok && ntile > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(ntile - 1) & 1],
                                              (uint32_t)((ntile - 1) >> 1) & 1u, abortp));
-    // The ring is idle once the last PV has landed: each 32-column slab of O
-    // is staged there ([128 heads][32 + 1 floats], padded against bank
-    // conflicts) and written out as whole 128-byte row segments.
-    float* stage = reinterpret_cast<float*>(ring);
-    constexpr int kStageLd = 33;
-    {  // all four softmax warps agree before the barriers below
+    {  // all four softmax warps agree before the named barriers below
       uint32_t all;
       asm volatile(
           "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
@@ -485,71 +485,225 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     if (ok) {
       tc_fence_after();
+      // Shared memory is idle once the last PV has landed (q's own half and
+      // the ring are one contiguous block).  It holds, for a split-KV merge,
+      // one other split's partial O (pbuf, in its global layout) and, for
+      // the output, the bf16 tile of this CTA's dims as kOCols / 64 TMA boxes
+      // of [128 heads][128 B], 128B-swizzled.
+      constexpr int kPartBytes = kAtHeads * kOCols * 4;
+      constexpr int kOutBoxes = kOCols / 64;
+      static_assert(kPartBytes + kOutBoxes * kAtSubBytes + 2 * kAtMaxSplits * kAtHeads * 4 <=
+                        Lay::kMiscOff,
+                    "epilogue buffers exceed the idle shared memory");
+      uint8_t* pbuf = base_ptr;
+      uint8_t* obuf = base_ptr + kPartBytes;
       const float sink_l2 = a.sink[head] * 1.4426950408889634f;
-      float scl = 1.f;
-      if (a.splits == 1) {
-        const float mm = fmaxf(m_run, sink_l2);
-        const float den = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - mm)) +
-                          exp2f(sink_l2 - mm);
-        scl = (m_run == -INFINITY || !(den > 0.f)) ? 0.f : exp2f(m_run - mm) / den;
-      } else {
-        const size_t unit = ((size_t)row_q * a.splits + split) * NQ + part;
-        float* pml = a.part_ml + unit * 2 * kAtHeads;
-        pml[head] = m_run;
-        pml[kAtHeads + head] = l_run;
-      }
+      const int S = a.splits;
+      const size_t unit0 = (size_t)row_q * S * NQ + part;  // unit of split s: unit0 + s * NQ
+      // Partial O layout per unit: [slab of 32 dims][16-byte unit u][head][4
+      // floats], so that a warp's 16-byte accesses at one (slab, u) are
+      // contiguous.
+      auto part_off = [&](int cc, int u) { return ((size_t)((cc / 32) * 8 + u) * kAtHeads + head) * 4; };
+      // One pass over the 32-column slabs.  Terms src * w, in split order:
+      // this CTA's O (TMEM; zero without tiles) and/or the partial in pbuf
+      // (`buf_first`: the pbuf term comes first).  acc = terms (`first`) or
+      // acc + terms, the running sum kept in TMEM columns [t_s, t_s +
+      // kOCols) (S and q are dead by now).  mode 0: acc back to TMEM; 1: out
+      // as this split's fp32 partial; 2: rotated back at -t, rounded to bf16
+      // and stored through TMA.  Every product and sum is rounded on its own,
+      // in split order, so a merge does not depend on which split performs
+      // it.
+      const uint32_t t_acc = t_s;
+      auto slab_pass = [&](bool use_own, float w_own, bool use_buf, float w_buf, bool buf_first,
+                           bool first, int mode) {
 #pragma unroll 1
-      for (int cc = 0; cc < kOCols; cc += 32) {
-        float o[32];
-        if (ntile > 0) {
-          uint32_t r[32];
-          tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
-          tmem_wait_ld();
+        for (int cc = 0; cc < kOCols; cc += 32) {
+          float o[32];
+          bool have = !first;
+          if (have) {
+            uint32_t r[32];
+            tmem_ld32(t_acc + lane_base + (uint32_t)cc, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(r[e]) * scl;
-        } else {
+            for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(r[e]);
+          }
+          auto add_own = [&]() {
+            uint32_t r[32];
+            if (ntile > 0) {
+              tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
+              tmem_wait_ld();
+            } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
-        }
-        if (a.splits == 1) {
-          const int d0 = part * kOCols + cc;
+              for (int e = 0; e < 32; ++e) r[e] = 0u;
+            }
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int d = d0 + e;
-            if (d >= rope0) {  // inverse rotation at -t
-              const int ii = (d - rope0) >> 1;
-              const float x0 = o[e], x1 = o[e + 1];
-              o[e] = x0 * sm.cs[ii] + x1 * sm.sn[ii];
-              o[e + 1] = -x0 * sm.sn[ii] + x1 * sm.cs[ii];
+            for (int e = 0; e < 32; ++e) {
+              const float tm = __fmul_rn(__uint_as_float(r[e]), w_own);
+              o[e] = have ? __fadd_rn(o[e], tm) : tm;
+            }
+            have = true;
+          };
+          auto add_buf = [&]() {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const float4 x =
+                  *reinterpret_cast<const float4*>(pbuf + part_off(cc, u) * sizeof(float));
+              const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const float tm = __fmul_rn(xs[v], w_buf);
+                o[4 * u + v] = have ? __fadd_rn(o[4 * u + v], tm) : tm;
+              }
+            }
+            have = true;
+          };
+          if (use_buf && buf_first) add_buf();
+          if (use_own) add_own();
+          if (use_buf && !buf_first) add_buf();
+          if (mode == 0) {
+            uint32_t w16[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(o[e]);
+            tmem_st16(t_acc + lane_base + (uint32_t)cc, w16);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(o[16 + e]);
+            tmem_st16(t_acc + lane_base + (uint32_t)cc + 16, w16);
+          } else if (mode == 1) {
+            float* dst = a.part_o + (unit0 + (size_t)split * NQ) * kAtHeads * kOCols;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<float4*>(dst + part_off(cc, u)) =
+                  make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+          } else {
+            const int d0 = part * kOCols + cc;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int d = d0 + e;
+              if (d >= rope0) {  // inverse rotation at -t
+                const int ii = (d - rope0) >> 1;
+                const float x0 = o[e], x1 = o[e + 1];
+                o[e] = x0 * sm.cs[ii] + x1 * sm.sn[ii];
+                o[e + 1] = -x0 * sm.sn[ii] + x1 * sm.cs[ii];
+              }
+            }
+            uint8_t* box = obuf + (cc / 64) * kAtSubBytes;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int u = ((cc & 63) >> 3) + j;
+              *reinterpret_cast<uint4*>(box + swz(head, u)) =
+                  make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
+                             pack_bf16x2(o[8 * j + 4], o[8 * j + 5]), pack_bf16x2(o[8 * j + 6], o[8 * j + 7]));
             }
           }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // previous slab written out
-#pragma unroll
-        for (int e = 0; e < 32; ++e) stage[head * kStageLd + e] = o[e];
+        if (mode == 0) {
+          tmem_wait_st();
+          tc_fence_before();
+        } else if (mode == 2) {
+          fence_proxy_async_shared();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (threadIdx.x == 0) {
+            for (int bx = 0; bx < kOutBoxes; ++bx)
+              tma_store_2d(&tm_out, obuf + bx * kAtSubBytes, part * kOCols + bx * 64,
+                           row_q * kAtHeads);
+            bulk_commit();
+            bulk_wait_read_all();
+          }
+        }
+      };
+      if (S == 1) {
+        const float mm = fmaxf(m_run, sink_l2);
+        const float den = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - mm)) +
+                          exp2f(sink_l2 - mm);
+        const float scl =
+            (m_run == -INFINITY || !(den > 0.f)) ? 0.f : exp2f(m_run - mm) / den;
+        slab_pass(true, scl, false, 0.f, false, true, 2);
+      } else {
+        // split-KV: publish (m, l, O) of this split; the last split of the
+        // (token, part) to finish merges all of them in split order (its
+        // own O straight from TMEM) and resets the arrival counter
+        float* pml = a.part_ml + (unit0 + (size_t)split * NQ) * 2 * kAtHeads;
+        pml[head] = m_run;
+        pml[kAtHeads + head] = l_run;
+        slab_pass(true, 1.f, false, 0.f, false, true, 1);
+        __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (a.splits == 1) {
-          // 128 rows x 64 B (bf16): 4 lanes per row, 16 B each
-          __nv_bfloat16* dst0 = a.out + (size_t)row_q * kAtHeads * kAtDim + part * kOCols + cc;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int rr = k * 32 + (threadIdx.x >> 2), q = threadIdx.x & 3;
-            const float* src = stage + rr * kStageLd + q * 8;
-            *reinterpret_cast<uint4*>(dst0 + (size_t)rr * kAtDim + q * 8) =
-                make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                           pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+        if (threadIdx.x == 0) {
+          const int old = atomicAdd(a.arrive + (size_t)row_q * NQ + part, 1);
+          sm.scan_tmp[0] = old == S - 1 ? 1 : 0;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (sm.scan_tmp[0]) {
+          __threadfence();
+          fence_proxy_async_global();  // the partials are read by bulk copies
+          // (m, l) of every split for this thread's head, in one batch of loads
+          float* mls = reinterpret_cast<float*>(obuf + kOutBoxes * kAtSubBytes);
+#pragma unroll 4
+          for (int sp = 0; sp < S; ++sp) {
+            const float* ml = a.part_ml + (unit0 + (size_t)sp * NQ) * 2 * kAtHeads;
+            mls[(2 * sp) * kAtHeads + head] = sp == split ? m_run : __ldcg(ml + head);
+            mls[(2 * sp + 1) * kAtHeads + head] = sp == split ? l_run : __ldcg(ml + kAtHeads + head);
           }
-        } else {
-          // 128 rows x 128 B (fp32): 8 lanes per row, 16 B each
-          const size_t unit = ((size_t)row_q * a.splits + split) * NQ + part;
-          float* dst0 = a.part_o + unit * kAtHeads * kOCols + cc;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int rr = k * 16 + (threadIdx.x >> 3), q = threadIdx.x & 7;
-            const float* src = stage + rr * kStageLd + q * 4;
-            *reinterpret_cast<float4*>(dst0 + (size_t)rr * kOCols + q * 4) =
-                make_float4(src[0], src[1], src[2], src[3]);
+          float M = sink_l2;
+          for (int sp = 0; sp < S; ++sp) M = fmaxf(M, mls[(2 * sp) * kAtHeads + head]);
+          float L = exp2f(sink_l2 - M);
+          for (int sp = 0; sp < S; ++sp) {
+            const float m = mls[(2 * sp) * kAtHeads + head];
+            if (m != -INFINITY) L += mls[(2 * sp + 1) * kAtHeads + head] * exp2f(m - M);
           }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          auto weight = [&](int sp) {
+            const float m = mls[(2 * sp) * kAtHeads + head];
+            return m == -INFINITY ? 0.f : exp2f(m - M) * inv;
+          };
+          int loads = 0;
+          bool okm = true;
+          auto fetch = [&](int sp) -> bool {  // partial O of split sp into pbuf
+            if (threadIdx.x == 0) {
+              mbar_arrive_expect_tx(&sm.merge_bar, kPartBytes);
+              bulk_load(pbuf, a.part_o + (unit0 + (size_t)sp * NQ) * kAtHeads * kOCols,
+                        kPartBytes, &sm.merge_bar);
+            }
+            bool got = __all_sync(0xffffffffu,
+                                  mbar_wait(&sm.merge_bar, (uint32_t)(loads & 1), abortp));
+            ++loads;
+            uint32_t all;  // the four warps agree before going on
+            asm volatile(
+                "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                : "=r"(all)
+                : "r"(got ? 1u : 0u)
+                : "memory");
+            return all != 0;
+          };
+          // passes over the splits in order; this CTA's own O joins the pass
+          // of its neighbour, so two splits take one pass and one copy
+          bool first = true;
+          for (int sp = 0; sp < S && okm;) {
+            if (sp == split) {
+              if (sp + 1 < S) {
+                okm = fetch(sp + 1);
+                if (!okm) break;
+                slab_pass(true, weight(sp), true, weight(sp + 1), false, first,
+                          sp + 2 == S ? 2 : 0);
+                sp += 2;
+              } else {
+                slab_pass(true, weight(sp), false, 0.f, false, first, 2);
+                sp += 1;
+              }
+            } else {
+              okm = fetch(sp);
+              if (!okm) break;
+              const bool with_own = sp + 1 == split;
+              const int next = sp + (with_own ? 2 : 1);
+              slab_pass(with_own, with_own ? weight(sp + 1) : 0.f, true, weight(sp), true, first,
+                        next == S ? 2 : 0);
+              sp = next;
+            }
+            first = false;
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // pbuf free again
+          }
+          if (threadIdx.x == 0) a.arrive[(size_t)row_q * NQ + part] = 0;
         }
       }
     }
@@ -698,79 +852,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
-  }
-}
-
-// Split-KV merge: per (query token, head, dim) the partials (m_s, l_s, O_s)
-// of every split, the sink and the inverse output rotation.  One block per
-// (query token, output part, 8 heads); a lane owns 512 / NQ / 32 consecutive
-// dims of one head.
-template <int NQ>
-__global__ void __launch_bounds__(256) k_attn_combine(AttnTcArgs a) {
-  constexpr int kOCols = kAtDim / NQ;
-  constexpr int kPer = kOCols / 32;  // 8 or 4
-  __shared__ float cs[kAtMaxRope / 2], sn[kAtMaxRope / 2];
-  const int row_q = blockIdx.x;
-  const int part = blockIdx.y;
-  const int head = blockIdx.z * 8 + (threadIdx.x >> 5);
-  const int c0 = (threadIdx.x & 31) * kPer;  // dims part * kOCols + c0 ..
-  const int t = a.q_pos[row_q];
-  const int rope0 = kAtDim - a.rope_dim;
-  const int S = a.splits;
-  if (threadIdx.x < a.rope_dim / 2) {
-    float c, s;
-    rope_cs_reduced(t, a.freq[threadIdx.x], &c, &s);
-    cs[threadIdx.x] = c;
-    sn[threadIdx.x] = s;
-  }
-  __syncthreads();
-  const float sink_l2 = a.sink[head] * 1.4426950408889634f;
-  float M = sink_l2;
-  for (int s = 0; s < S; ++s) {
-    const size_t unit = ((size_t)row_q * S + s) * NQ + part;
-    M = fmaxf(M, a.part_ml[unit * 2 * kAtHeads + head]);
-  }
-  float L = exp2f(sink_l2 - M);
-  float o[kPer];
-#pragma unroll
-  for (int e = 0; e < kPer; ++e) o[e] = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const size_t unit = ((size_t)row_q * S + s) * NQ + part;
-    const float m = a.part_ml[unit * 2 * kAtHeads + head];
-    if (m == -INFINITY) continue;
-    const float w = exp2f(m - M);
-    L += a.part_ml[unit * 2 * kAtHeads + kAtHeads + head] * w;
-    const float4* src =
-        reinterpret_cast<const float4*>(a.part_o + (unit * kAtHeads + head) * kOCols + c0);
-#pragma unroll
-    for (int q4 = 0; q4 < kPer / 4; ++q4) {
-      const float4 v = src[q4];
-      o[4 * q4] += v.x * w;
-      o[4 * q4 + 1] += v.y * w;
-      o[4 * q4 + 2] += v.z * w;
-      o[4 * q4 + 3] += v.w * w;
-    }
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-  for (int e = 0; e < kPer; e += 2) {
-    float x0 = o[e] * inv, x1 = o[e + 1] * inv;
-    const int d = part * kOCols + c0 + e;
-    if (d >= rope0) {  // inverse rotation at -t
-      const float c = cs[(d - rope0) >> 1], s = sn[(d - rope0) >> 1];
-      const float y0 = x0 * c + x1 * s, y1 = -x0 * s + x1 * c;
-      x0 = y0;
-      x1 = y1;
-    }
-    o[e] = x0;
-    o[e + 1] = x1;
-  }
-  __nv_bfloat16* dst = a.out + ((size_t)row_q * kAtHeads + head) * kAtDim + part * kOCols + c0;
-  if (kPer == 8) {
-    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                                pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
-  } else {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
   }
 }
 

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -117,9 +118,12 @@ csa_status_t check_sizes(int B, int Tq, int n_max) {
   return CSA_OK;
 }
 
+std::atomic<unsigned long long> g_launches{0};
+
 csa_status_t launched(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return CSA_OK;
 }
 
@@ -196,27 +200,44 @@ size_t scores_bytes(int B, int Tq, int n_max) {
   return round_up((size_t)B * Tq * (size_t)n_max * sizeof(float), 256);
 }
 
-// Top-k plan: one block per row (candidates in registers) up to 16384
-// entries; two stages (per-chunk top-k, then a merge of the candidates) up to
-// 16 chunks of 16384 when the merge fits one block; else the generic
-// shared-memory radix select.
-constexpr int kTopkChunk = 1024 * 16;
-int topk_chunks(const csa_params_t* p, int n_max) {
-  if (n_max <= kTopkChunk) return 1;
-  const int c = (n_max + kTopkChunk - 1) / kTopkChunk;
-  if (c <= 64 && (long long)c * p->topk <= kTopkChunk) return c;
-  return 0;  // generic path
+// Top-k plan.  A block holds its candidates in registers: 2048 (256 x 8) or
+// 16384 (1024 x 16) entries.  One block per row when the row fits; two
+// stages (per-chunk top-k into a candidate list, then one merge block per
+// row over the concatenated candidates) for longer rows when the merge fits
+// one block (4096, 8192 or 16384 candidates); else the generic
+// shared-memory radix select.  (Splitting rows that fit one block over more
+// chunks, to occupy more SMs when rows are few, measured slower: a block's
+// select costs about the same for 4096 entries as for 16384.)
+struct TopkPlan {
+  int chunks;     // 0: generic; 1: single stage; >1: chunk + merge
+  int chunk_len;  // entries per chunk block
+  int merge_cap;  // candidates per merge block
+};
+constexpr int kTopkSmall = 256 * 8, kTopkMid = 256 * 16, kTopkBig = 1024 * 16;
+
+TopkPlan topk_plan(const csa_params_t* p, int B, int Tq, int n_max) {
+  (void)B;
+  (void)Tq;
+  const long long k = p->topk;
+  if (n_max <= kTopkSmall) return {1, kTopkSmall, 0};
+  if (n_max <= kTopkBig) return {1, kTopkBig, 0};
+  const long long c = (n_max + kTopkBig - 1) / kTopkBig;
+  if (c <= 64 && c * k <= kTopkBig) {
+    const long long cand = c * k;
+    return {(int)c, kTopkBig,
+            cand <= kTopkMid ? kTopkMid : (cand <= 2 * kTopkMid ? 2 * kTopkMid : kTopkBig)};
+  }
+  return {0, 0, 0};
 }
 
 size_t topk_ws_bytes(const csa_params_t* p, int B, int Tq, int n_max) {
-  const int c = topk_chunks(p, n_max);
+  const int c = topk_plan(p, B, Tq, n_max).chunks;
   if (c <= 1) return 0;
   const size_t rows = (size_t)B * Tq;
   return round_up(rows * c * (size_t)p->topk * sizeof(int), 256) +
          round_up(rows * c * sizeof(int), 256);
 }
 
-int num_sms();
 
 // Tensor-core attention applies to the measured head shape in bf16.
 bool attn_tc_ok(const csa_params_t* p, csa_dtype_t dtype, bool hca, int n_max) {
@@ -240,7 +261,7 @@ int attn_splits(const csa_params_t* p, bool hca, int B, int Tq, int n_max) {
   long long s = num_sms() / units;
   const long long max_s = (rows + kAtTile - 1) / kAtTile;
   if (s > max_s) s = max_s;
-  if (s > 32) s = 32;
+  if (s > kAtMaxSplits) s = kAtMaxSplits;
   return s < 1 ? 1 : (int)s;
 }
 
@@ -251,7 +272,8 @@ size_t attn_ws_bytes(const csa_params_t* p, csa_dtype_t dtype, bool hca, int B, 
   if (sp == 1) return 0;
   const size_t units = (size_t)B * Tq * sp * attn_nq(B, Tq);
   return round_up(units * kAtHeads * (kAtDim / attn_nq(B, Tq)) * sizeof(float), 256) +
-         round_up(units * 2 * kAtHeads * sizeof(float), 256);
+         round_up(units * 2 * kAtHeads * sizeof(float), 256) +
+         round_up((size_t)B * Tq * attn_nq(B, Tq) * sizeof(int), 256);
 }
 
 }  // namespace
@@ -279,6 +301,10 @@ CSA_API const char* csa_status_string(csa_status_t s) {
 }
 
 CSA_API const char* csa_last_error_detail(void) { return g_detail; }
+
+CSA_API uint64_t csa_launch_count(void) {
+  return g_launches.load(std::memory_order_relaxed);
+}
 
 CSA_API csa_status_t csa_workspace_size(const csa_params_t* p, csa_op_t op, int32_t B, int32_t Tq,
                                 int32_t n_max, size_t* bytes) {
@@ -392,9 +418,10 @@ static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const 
                               int32_t* idx_out, void* ws, size_t ws_bytes, cudaStream_t s) {
   const unsigned rows = (unsigned)B * (unsigned)Tq;
   const int k = p->topk;
-  const int chunks = topk_chunks(p, n_max);
+  const TopkPlan plan = topk_plan(p, B, Tq, n_max);
+  const int chunks = plan.chunks;
   if (chunks == 1) {
-    if (n_max <= 2048)
+    if (plan.chunk_len == kTopkSmall)
       k_topk_chunk<256, 8><<<dim3(1, rows), 256, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k,
                                                           p->width, p->stride, 1, idx_out,
                                                           nullptr, nullptr);
@@ -415,7 +442,13 @@ static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const 
     k_topk_chunk<1024, 16><<<dim3((unsigned)chunks, rows), 1024, 0, s>>>(
         scores, q_pos, n_cmp, Tq, n_max, k, p->width, p->stride, chunks, idx_out, cand, cand_n);
     CSA_CHECK(launched("k_topk_chunk"));
-    k_topk_merge<1024, 16><<<rows, 1024, 0, s>>>(scores, n_max, k, chunks, cand, cand_n, idx_out);
+    if (plan.merge_cap == kTopkMid)
+      k_topk_merge<256, 16><<<rows, 256, 0, s>>>(scores, n_max, k, chunks, cand, cand_n, idx_out);
+    else if (plan.merge_cap == 2 * kTopkMid)
+      k_topk_merge<512, 16><<<rows, 512, 0, s>>>(scores, n_max, k, chunks, cand, cand_n, idx_out);
+    else
+      k_topk_merge<1024, 16><<<rows, 1024, 0, s>>>(scores, n_max, k, chunks, cand, cand_n,
+                                                   idx_out);
     return launched("k_topk_merge");
   }
   k_topk_rows<1024><<<rows, 1024, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k, p->width,
@@ -530,23 +563,25 @@ static csa_status_t launch_attn_simt(const AttnArgs& a, csa_dtype_t dtype, cudaS
 
 template <bool kHca, int NQ>
 static csa_status_t launch_attn_tc_nq(const AttnArgs& g, AttnTcArgs& a, int sp, void* ws,
-                                      const CUtensorMap& tq, cudaStream_t s) {
+                                      const CUtensorMap& tq, const CUtensorMap& to,
+                                      cudaStream_t s) {
   using Lay = AtLayout<NQ>;
   if (sp > 1) {
+    // workspace: partial O | partial (m, l) | arrival counters (zeroed here)
     const size_t units = (size_t)g.B * g.Tq * sp * NQ;
+    const size_t o_bytes = round_up(units * kAtHeads * (kAtDim / NQ) * sizeof(float), 256);
+    const size_t ml_bytes = round_up(units * 2 * kAtHeads * sizeof(float), 256);
     a.part_o = (float*)ws;
-    a.part_ml = (float*)((char*)ws + round_up(units * kAtHeads * (kAtDim / NQ) * sizeof(float), 256));
+    a.part_ml = (float*)((char*)ws + o_bytes);
+    a.arrive = (int*)((char*)ws + o_bytes + ml_bytes);
+    if (cudaMemsetAsync(a.arrive, 0, (size_t)g.B * g.Tq * NQ * sizeof(int), s) != cudaSuccess)
+      return fail(CSA_ERR_CUDA, "cudaMemsetAsync of the split counters failed");
   }
   const size_t smem = Lay::kBytes + 1024;
   CSA_CHECK(set_smem_attr(k_attn_tc<kHca, NQ>, smem, "k_attn_tc"));
   dim3 grid((unsigned)(NQ * sp), (unsigned)(g.B * g.Tq));
-  k_attn_tc<kHca, NQ><<<grid, kAtThreads, smem, s>>>(a, tq);
-  CSA_CHECK(launched("k_attn_tc"));
-  if (sp > 1) {
-    k_attn_combine<NQ><<<dim3((unsigned)(g.B * g.Tq), NQ, kAtHeads / 8), 256, 0, s>>>(a);
-    CSA_CHECK(launched("k_attn_combine"));
-  }
-  return CSA_OK;
+  k_attn_tc<kHca, NQ><<<grid, kAtThreads, smem, s>>>(a, tq, to);
+  return launched("k_attn_tc");
 }
 
 template <bool kHca>
@@ -580,12 +615,14 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   a.out = (__nv_bfloat16*)g.out;
   a.part_o = nullptr;
   a.part_ml = nullptr;
+  a.arrive = nullptr;
   for (int i = 0; i < kAtMaxRope / 2; ++i)
     a.freq[i] = i < g.rope_dim / 2 ? std::pow(g.theta, -2.0 * i / (double)g.rope_dim) : 0.0;
-  CUtensorMap tq;
+  CUtensorMap tq, to;
   CSA_CHECK(make_tmap_bf16(&tq, g.q, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
-  if (attn_nq(g.B, g.Tq) == 4) return launch_attn_tc_nq<kHca, 4>(g, a, sp, ws, tq, s);
-  return launch_attn_tc_nq<kHca, 2>(g, a, sp, ws, tq, s);
+  CSA_CHECK(make_tmap_bf16(&to, g.out, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
+  if (attn_nq(g.B, g.Tq) == 4) return launch_attn_tc_nq<kHca, 4>(g, a, sp, ws, tq, to, s);
+  return launch_attn_tc_nq<kHca, 2>(g, a, sp, ws, tq, to, s);
 }
 
 static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32_t* q_pos,

@@ -1,12 +1,14 @@
 // Step 2b, fast path: exact top-k ("keeps the top 1,024 entries") of one
 // query row held in registers, ties to the lower index, output ascending.
 //
-// Each of NT threads owns PT consecutive candidates (so thread order then
-// register order is index order).  Radix select on order-preserving uint32
-// keys, 8 bits per pass, starting at the highest bit in which the row's keys
-// differ.  After the last pass the threshold key T and the number of keys
-// equal to T to keep are exact; one pair of block-wide scans over per-thread
-// counts then places every kept index.
+// Each of NT threads holds PT candidates, striped: candidate slot e of thread
+// t is position e * NT + t of the block's range, so the loads coalesce.
+// Radix select on order-preserving uint32 keys, 8 bits per pass, starting at
+// the highest bit in which the row's keys differ, and stopping as soon as
+// the bin that holds the k-th key is taken whole.  Then the kept candidates
+// are placed in index order: per (slot, warp) ballots give counts, one
+// block scan over those counts (slot-major, then warp) gives each group's
+// first output position.
 //
 // Rows longer than one block's capacity use two stages: each chunk keeps its
 // own top-k (k_topk_chunk), then the candidates of all chunks, in index
@@ -18,32 +20,67 @@
 
 namespace csa {
 
+template <int NT, int PT>
 struct TopkShared {
+  static constexpr int kGroups = PT * (NT / 32);  // (slot, warp) groups in index order
   unsigned hist[256];
   int scan[33];
   uint32_t prefix;
   int remaining;
+  int bin_count;
   uint32_t red_and[32], red_or[32];
+  int cnt[kGroups];
 };
 
-// Exclusive block scan of one int per thread (also returns the total).
-__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total) {
-  return block_inclusive_scan(v, tmp, total) - v;
+// Exclusive scan, in place, of the kGroups counts in sh.cnt (every thread
+// calls it; the counts must have been written before).  Returns the total.
+template <int NT, int PT>
+__device__ __forceinline__ int scan_groups(TopkShared<NT, PT>& sh) {
+  constexpr int G = TopkShared<NT, PT>::kGroups;
+  static_assert(G <= NT, "one thread per group");
+  __syncthreads();
+  const int v = (int)threadIdx.x < G ? sh.cnt[threadIdx.x] : 0;
+  int total;
+  const int incl = block_inclusive_scan(v, sh.scan, &total);
+  if ((int)threadIdx.x < G) sh.cnt[threadIdx.x] = incl - v;
+  __syncthreads();
+  return total;
+}
+
+// Writes index_of(e) of every selected candidate to out[position] (positions
+// in index order, only those below k); returns the number selected.
+template <int NT, int PT, typename IndexOf>
+__device__ __forceinline__ int place_selected(const bool (&sel)[PT], int k, IndexOf index_of,
+                                              int* out, TopkShared<NT, PT>& sh) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  unsigned m[PT];
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    m[e] = __ballot_sync(0xffffffffu, sel[e]);
+    if (lane == 0) sh.cnt[e * NW + wid] = __popc(m[e]);
+  }
+  const int total = scan_groups(sh);
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    if (sel[e]) {
+      const int pos = sh.cnt[e * NW + wid] + __popc(m[e] & lt);
+      if (pos < k) out[pos] = index_of(e);
+    }
+  }
+  return total;
 }
 
 // Selects the top `k` of the block's candidates.  key[e], valid[e] describe
-// candidate thread*PT + e; index_of(e) gives its output index.  Writes the
-// kept indices, ascending, to out[0 .. min(k, n_valid)) and returns that
-// count (same value in every thread).
-//
-// The radix passes start at the highest bit in which the valid keys differ
-// (a block AND/OR reduction finds it), so the first digit already spreads
-// over many bins; digits are 8 bits wide from there down to bit 0.  Each
-// pass picks its digit with a 256-thread suffix scan over the histogram.
+// candidate slot e (position e * NT + threadIdx.x); index_of(e) gives its
+// output index.  Writes the kept indices, ascending, to out[0 .. min(k,
+// n_valid)) and returns that count (same value in every thread).
 template <int NT, int PT, typename IndexOf>
 __device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], int k,
-                          IndexOf index_of, int* out, TopkShared& sh) {
+                          IndexOf index_of, int* out, TopkShared<NT, PT>& sh) {
   static_assert(NT >= 256, "bin scan needs 256 threads");
+  constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int nv_local = 0;
   uint32_t k_and = 0xffffffffu, k_or = 0u;
@@ -56,14 +93,8 @@ __device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], in
     }
   }
   int n_valid;
-  const int before = block_exclusive_scan(nv_local, sh.scan, &n_valid);
-  if (n_valid <= k) {  // keep every valid candidate
-    int p = before;
-#pragma unroll
-    for (int e = 0; e < PT; ++e)
-      if (valid[e]) out[p++] = index_of(e);
-    return n_valid;
-  }
+  block_inclusive_scan(nv_local, sh.scan, &n_valid);
+  if (n_valid <= k) return place_selected<NT, PT>(valid, k, index_of, out, sh);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     k_and &= __shfl_xor_sync(0xffffffffu, k_and, o);
@@ -76,7 +107,7 @@ __device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], in
   __syncthreads();
   k_and = 0xffffffffu;
   k_or = 0u;
-  for (int w = 0; w < NT / 32; ++w) {
+  for (int w = 0; w < NW; ++w) {
     k_and &= sh.red_and[w];
     k_or |= sh.red_or[w];
   }
@@ -85,6 +116,7 @@ __device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], in
   int remaining = k;
   if (diff == 0u) {  // all valid keys equal
     prefix = k_and;
+    mask = 0xffffffffu;
   } else {
     int hi = 31 - __clz(diff);
     mask = hi == 31 ? 0u : (0xffffffffu << (hi + 1));  // bits above hi are common
@@ -119,6 +151,7 @@ __device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], in
         if (incl >= remaining && excl < remaining) {
           sh.prefix = prefix | ((uint32_t)bin << lo);
           sh.remaining = remaining - excl;
+          sh.bin_count = h;
         }
       }
       __syncthreads();
@@ -126,32 +159,29 @@ __device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], in
       remaining = sh.remaining;
       mask |= dmask << lo;
       hi = lo - 1;
+      if (remaining == sh.bin_count) break;  // the boundary bin is kept whole
     }
   }
-  const uint32_t thr = prefix;
-  const int take_eq = remaining;
-  int gt = 0, eq = 0;
+  // kept: keys above the boundary bin, and the first `remaining` keys (in
+  // index order) of the boundary bin
+  bool gt[PT], eq[PT];
+  unsigned meq[PT];
 #pragma unroll
   for (int e = 0; e < PT; ++e) {
-    gt += (valid[e] && key[e] > thr) ? 1 : 0;
-    eq += (valid[e] && key[e] == thr) ? 1 : 0;
+    const uint32_t km = key[e] & mask;
+    gt[e] = valid[e] && km > prefix;
+    eq[e] = valid[e] && km == prefix;
+    meq[e] = __ballot_sync(0xffffffffu, eq[e]);
+    if (lane == 0) sh.cnt[e * NW + wid] = __popc(meq[e]);
   }
-  int eq_tot;
-  const int eq_before = block_exclusive_scan(eq, sh.scan, &eq_tot);
-  const int my_eq = max(0, min(eq, take_eq - eq_before));
-  int sel_tot;
-  int pos = block_exclusive_scan(gt + my_eq, sh.scan, &sel_tot);
-  int eq_taken = 0;
+  scan_groups(sh);
+  const unsigned lt = (1u << lane) - 1u;
+  bool sel[PT];
 #pragma unroll
-  for (int e = 0; e < PT; ++e) {
-    if (!valid[e]) continue;
-    bool take = key[e] > thr;
-    if (!take && key[e] == thr && eq_taken < my_eq) {
-      take = true;
-      ++eq_taken;
-    }
-    if (take && pos < k) out[pos++] = index_of(e);
-  }
+  for (int e = 0; e < PT; ++e)
+    sel[e] = gt[e] || (eq[e] && sh.cnt[e * NW + wid] + __popc(meq[e] & lt) < remaining);
+  __syncthreads();  // every thread has read the tie ranks before cnt is reused
+  place_selected<NT, PT>(sel, k, index_of, out, sh);
   return k;
 }
 
@@ -165,23 +195,22 @@ __global__ void __launch_bounds__(NT)
                  const int* __restrict__ n_cmp, int Tq, int n_max, int k, int width, int stride,
                  int n_chunks, int* __restrict__ idx_out, int* __restrict__ cand,
                  int* __restrict__ cand_n) {
-  __shared__ TopkShared sh;
+  __shared__ TopkShared<NT, PT> sh;
   const int c = blockIdx.x, row = blockIdx.y;
   const int b = row / Tq;
   const int nv = min(n_visible(q_pos[row], n_cmp[b], width, stride), n_max);
-  const int base = c * NT * PT;
+  const int base = c * NT * PT + (int)threadIdx.x;
   const float* s = scores + (size_t)row * n_max;
   uint32_t key[PT];
   bool valid[PT];
-  const int first = base + threadIdx.x * PT;
 #pragma unroll
   for (int e = 0; e < PT; ++e) {
-    const int j = first + e;
+    const int j = base + e * NT;
     valid[e] = j < nv;
     key[e] = valid[e] ? float_key(s[j]) : 0u;
   }
   int* out = n_chunks == 1 ? idx_out + (size_t)row * k : cand + ((size_t)row * n_chunks + c) * k;
-  const int cnt = block_topk<NT, PT>(key, valid, k, [&](int e) { return first + e; }, out, sh);
+  const int cnt = block_topk<NT, PT>(key, valid, k, [&](int e) { return base + e * NT; }, out, sh);
   if (n_chunks == 1) {
     for (int i = cnt + threadIdx.x; i < k; i += NT) out[i] = -1;
   } else if (threadIdx.x == 0) {
@@ -195,7 +224,7 @@ __global__ void __launch_bounds__(NT)
     k_topk_merge(const float* __restrict__ scores, int n_max, int k, int n_chunks,
                  const int* __restrict__ cand, const int* __restrict__ cand_n,
                  int* __restrict__ idx_out) {
-  __shared__ TopkShared sh;
+  __shared__ TopkShared<NT, PT> sh;
   __shared__ int offs[65];
   const int row = blockIdx.x;
   if (threadIdx.x == 0) {
@@ -212,16 +241,18 @@ __global__ void __launch_bounds__(NT)
   uint32_t key[PT];
   bool valid[PT];
   int idx[PT];
-  const int first = threadIdx.x * PT;
-  int c = 0;
 #pragma unroll
   for (int e = 0; e < PT; ++e) {
-    const int p = first + e;
+    const int p = e * NT + (int)threadIdx.x;
     valid[e] = p < total;
     idx[e] = -1;
     if (valid[e]) {
-      while (c + 1 < n_chunks && offs[c + 1] <= p) ++c;
-      idx[e] = cand[((size_t)row * n_chunks + c) * k + (p - offs[c])];
+      int lo = 0, hi = n_chunks - 1;  // last chunk c with offs[c] <= p
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offs[mid] <= p) lo = mid; else hi = mid - 1;
+      }
+      idx[e] = cand[((size_t)row * n_chunks + lo) * k + (p - offs[lo])];
     }
     key[e] = valid[e] ? float_key(s[idx[e]]) : 0u;
   }

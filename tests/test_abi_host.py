@@ -40,6 +40,13 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def test_launch_counter_counts_no_rejected_call(lib):
+    before = csa.csa_launch_count()
+    with pytest.raises(csa.CsaError):
+        csa.csa_workspace_size(csa.Params(d=100), csa.CSA_OP_INDEX_TOPK, 1, 1, 10)
+    assert csa.csa_launch_count() == before
+
+
 def test_abi_version_and_status_strings(lib):
     assert lib.csa_abi_version() == 1
     for code, name in L.STATUS.items():

@@ -13,7 +13,8 @@ import torch
 
 import oracle
 from gpu_util import assert_close, dev, f64, host64, params_of, run_decode, run_hca, run_prefill
-from sparse_compressed_attention_csa_b200 import (CSA_OP_SPARSE_ATTN, CsaError, Params,
+from sparse_compressed_attention_csa_b200 import (CSA_OP_SPARSE_ATTN, CSA_OP_TOPK_SELECT,
+                                                  CsaError, Params,
                                                   csa_compress, csa_workspace_size,
                                                   csa_index_scores, csa_poll_device_error,
                                                   csa_sparse_attn, csa_topk_select, layer)
@@ -134,6 +135,7 @@ def test_prefill_small_heads_f32():
 def test_hca_ragged_and_early_queries():
     check_hca(W.HCA_DECODE_128K.replace(B=3, T=1000, seed=25))   # N = 7
     check_hca(W.HCA_DECODE_128K.replace(B=2, T=100, seed=26))    # N = 0: window + sink only
+    check_hca(W.HCA_DECODE_128K.replace(B=2, T=3, seed=27))      # one split holds no rows
 
 
 def test_compress_hca_width_bf16_and_f32():
@@ -166,10 +168,8 @@ def test_index_scores_bit_exact():
         assert np.array_equal(got[tq, :nv], want[tq, :nv]), tq
 
 
-def test_topk_select_adversarial_scores():
-    rng = np.random.default_rng(29)
-    n, k = 5000, 1024
-    cases = [
+def _adversarial_rows(rng, n):
+    return [
         np.zeros(n),                                        # all tied
         np.where(rng.random(n) < 0.5, 0.0, -0.0),           # signed zeros tie
         rng.integers(0, 3, n).astype(np.float64),           # few distinct values
@@ -178,13 +178,29 @@ def test_topk_select_adversarial_scores():
         np.concatenate([np.full(n // 2, 7.0), rng.random(n - n // 2)]),
         rng.standard_normal(n).astype(np.float32).astype(np.float64),
     ]
-    scores = np.stack(cases).astype(np.float32)[:, None, :]     # [B, 1, n]
+
+
+# (entries, k, rows): one block per row up to 16384 entries, else chunks of
+# 16384 and a merge block of 4096, 8192 or 16384 candidates
+@pytest.mark.parametrize("n,k,rows", [
+    (5000, 1024, 7),      # one 16384-entry block per row
+    (1500, 64, 20),       # one 2048-entry block per row
+    (40000, 1024, 7),     # 3 chunks, merge of 3072 candidates
+    (70000, 1024, 7),     # 5 chunks, merge of 5120
+    (70000, 3000, 3),     # 5 chunks, merge of 15000
+])
+def test_topk_select_adversarial_scores(n, k, rows):
+    rng = np.random.default_rng(29 + n + k + rows)
+    base = _adversarial_rows(rng, n)
+    scores = np.stack([base[r % len(base)] for r in range(rows)]).astype(np.float32)[:, None, :]
     B = scores.shape[0]
     p = Params(topk=k, width=8, stride=4)
     q_pos = np.full((B, 1), 4 * (n - 1) + 7, dtype=np.int32)   # every entry visible
     n_cmp = np.full((B,), n, dtype=np.int32)
     idx = torch.empty((B, 1, k), dtype=torch.int32, device="cuda")
-    csa_topk_select(p, dev(scores), dev(q_pos), dev(n_cmp), idx)
+    nb = csa_workspace_size(p, CSA_OP_TOPK_SELECT, B, 1, n)
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device="cuda")
+    csa_topk_select(p, dev(scores), dev(q_pos), dev(n_cmp), idx, ws)
     torch.cuda.synchronize()
     got = idx.cpu().numpy()
     for b in range(B):
