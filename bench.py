@@ -1,21 +1,27 @@
 #!/usr/bin/env python
-"""Benchmark of the CSA decode layer on B200: query-heads/s at 64K context,
-batch 32 (one layer: lightning indexer + exact top-1024 + sparse shared-KV
-attention over 1,024 selected entries and a 128-token window).
+"""Benchmark of the CSA layer on B200.
+
+Headline: CSA decode at 64K context, batch 32 (one layer: lightning indexer
++ exact top-1024 + sparse shared-KV attention over 1,024 selected entries
+and a 128-token window), in query-heads/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload NAME]
 
-One step = the whole decode hot path over one batch (32 sequences x 1 query
-token x 128 heads) with the caches resident in HBM.  Each rank runs an
-independent replica of the workload (replicas only: the decode batch
-shards with no exchange), so `scaling` is weak and `value` sums all ranks'
-query-heads over the slowest rank's time.  L2 is flushed before every timed
-step (a 256 MiB write, then a 256 MiB read, so that no dirty line of the
-flush is left for the step to write back); each step is a captured CUDA graph
-whose per-kernel durations come from CUDA events recorded inside it.
+One step = the whole hot path over one batch with the inputs resident in HBM:
+decode: indexer scores -> top-k -> sparse attention; HCA decode: dense
+attention over every compressed entry; prefill: compression -> indexer ->
+top-k -> attention for every token.  Each rank runs an independent replica
+of the workload (replicas only: the batch shards with no exchange), so
+`scaling` is weak and `value` sums all ranks' query-heads over the slowest
+rank's time.  L2 is flushed before every timed step (a 256 MiB write, then a
+256 MiB read, so that no dirty line of the flush is left for the step to
+write back).  The step runs as one captured CUDA graph timed with CUDA events
+on its stream; the per-kernel breakdown comes from a second graph with
+events between the launches.
 
 `--impl reference` times the fp64 CPU oracle (the only other place this file
-runs it) on the host cores, one sequence per step.
+runs it) on the host cores, on a bounded sample of the workload per step.
 """
 from __future__ import annotations
 
@@ -30,37 +36,12 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+HEADLINE = "csa_decode_bs32_ctx65536"
 METRIC = "CSA decode query-heads/s at 64K ctx bs32; % of HBM / bf16 tensor roofline"
 UNIT = "query-heads/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_csa_decode_bs32_ctx65536.json")
-
-
-def _source_digest():
-    """Digest of the kernel sources: recorded DRAM traffic is only reported
-    for the kernels it was captured from."""
-    import hashlib
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "sparse_compressed_attention_csa_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(f.encode())
-            h.update(open(os.path.join(csrc, f), "rb").read())
-    return h.hexdigest()[:16]
-
-
-def _recorded_traffic(wl):
-    """DRAM bytes per launch group (dram__bytes_read.sum + dram__bytes_write.sum
-    from one ncu capture of this workload), or {} if the kernels changed."""
-    try:
-        rec = json.load(open(TRAFFIC_FILE))
-    except (OSError, ValueError):
-        return {}
-    if rec.get("source_digest") != _source_digest() or rec.get("workload") != wl.name:
-        return {}
-    return {k: v for k, v in rec.get("bytes_per_launch", {}).items()}
 
 
 def _args():
@@ -69,6 +50,14 @@ def _args():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
+    ap.add_argument("--workload", default=HEADLINE,
+                    help="csa_decode_bs32_ctx65536 (default), csa_decode_bs4_ctx1048576, "
+                         "hca_decode_bs16_ctx131072 or csa_prefill_T8192")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--flush-mib", type=int, default=256,
+                    help="L2 flush size per side (0: no flush; only for profiling, where the "
+                         "profiler flushes caches itself)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
@@ -76,40 +65,76 @@ def _args():
     return a
 
 
-def _workload():
+def _workload(name, batch=0):
     from sparse_compressed_attention_csa_b200 import workloads as W
-    return W.CSA_DECODE_64K
+    if name not in W.WORKLOADS or W.WORKLOADS[name].dtype != "bf16":
+        raise SystemExit(f"unknown workload {name}; choose from "
+                         f"{[n for n, w in W.WORKLOADS.items() if w.dtype == 'bf16']}")
+    wl = W.WORKLOADS[name]
+    if batch and batch != wl.B:
+        wl = wl.replace(B=batch, name=f"{name}_b{batch}")
+    return wl
 
 
-def _config(wl, extra=None):
-    c = {"workload": wl.name, "batch": wl.B, "context": wl.T, "n_cmp": wl.n_cmp,
-         "query_heads": wl.n_heads, "head_dim": wl.d, "rope_dim": wl.rope_dim,
-         "indexer": f"{wl.idx_heads}x{wl.idx_dim}", "topk": wl.topk, "window": wl.window,
-         "l2": "flushed before every timed step: 256 MiB write, then 256 MiB read (L2 left clean)",
+def _metric(wl):
+    return METRIC if wl.name == HEADLINE else f"{wl.name} query-heads/s"
+
+
+def _config(wl, extra=None, flush_mib=256):
+    c = {"workload": wl.name, "kind": wl.kind, "batch": wl.B, "context": wl.T,
+         "n_cmp": wl.n_cmp, "query_tokens_per_seq": wl.Tq, "query_heads": wl.n_heads,
+         "head_dim": wl.d, "rope_dim": wl.rope_dim, "pool": f"{wl.width}/stride {wl.stride}",
+         "window": wl.window,
+         "l2": (f"flushed before every timed step: {flush_mib} MiB write, then {flush_mib} MiB read "
+                "(L2 left clean)") if flush_mib else "not flushed",
          "parallelism": "replicas"}
+    if wl.kind != "hca_decode":
+        c.update({"indexer": f"{wl.idx_heads}x{wl.idx_dim}", "topk": wl.topk})
     if extra:
         c.update(extra)
     return c
 
 
 def algorithmic_work(wl):
-    """Bytes (and FLOPs) one decode step must move (do) at least, per kernel
-    group and for the whole step, with the caches resident in HBM."""
-    B, N, H, d = wl.B, wl.n_cmp, wl.n_heads, wl.d
+    """Bytes (and FLOPs) each kernel group of one step must move (do) at
+    least, with the inputs resident in HBM, and the whole step's bytes."""
+    B, N, H, d, T = wl.B, wl.n_cmp, wl.n_heads, wl.d, wl.T
+    Tq = wl.Tq
+    n_q = B * Tq
+    q = n_q * H * d * 2
+    out = n_q * H * d * 2
+    if wl.kind == "hca_decode":
+        rows = n_q * (N + wl.window) * d * 2
+        g = {"hca_attn": {"bytes": rows + q + out + H * 4,
+                          "flops": 4 * n_q * H * (N + wl.window) * d}}
+        g["step"] = {"bytes": g["hca_attn"]["bytes"]}
+        return g
     keys = B * N * wl.idx_dim * 2
-    idx_q = B * wl.idx_heads * wl.idx_dim * 2 + B * wl.idx_heads * 4
-    scores = B * N * 4
-    sel = B * wl.topk * 4
-    n_rows = min(wl.topk, N) + wl.window
-    rows = B * n_rows * d * 2
-    q = B * H * d * 2
-    out = B * H * d * 2
-    return {
-        "index_scores": {"bytes": keys + idx_q + scores, "flops": 2 * B * N * wl.idx_heads * wl.idx_dim},
-        "topk_select": {"bytes": scores + sel, "flops": 0},
-        "sparse_attn": {"bytes": rows + q + out + sel + H * 4, "flops": 4 * B * H * n_rows * d},
-        "step": {"bytes": keys + idx_q + rows + q + out + sel + H * 4},
-    }
+    idx_q = n_q * wl.idx_heads * (wl.idx_dim * 2 + 4)
+    if wl.kind == "csa_decode":
+        vis = N                      # every entry is visible to the decode query
+        n_rows = min(wl.topk, N) + wl.window
+        rows = n_q * n_rows * d * 2  # gathered rows (selected + window)
+        pre = {}
+    else:
+        # causal prefill: query t sees floor((t - width) / stride) + 1 entries
+        vis = sum(max(0, (t - wl.width) // wl.stride + 1) for t in range(T)) / T
+        n_rows = sum(min(wl.topk, max(0, (t - wl.width) // wl.stride + 1)) +
+                     min(wl.window, t + 1) for t in range(T)) / T
+        rows = B * (N + T) * d * 2   # every pooled entry and raw row read once
+        pre = {"compress": {"bytes": B * T * d * 2 * 2 + B * N * d * 2 + B * T * d * 2,
+                            "flops": 0}}
+    scores = int(n_q * vis) * 4
+    sel = n_q * wl.topk * 4
+    g = dict(pre)
+    g["index_scores"] = {"bytes": keys + idx_q + scores,
+                         "flops": int(2 * n_q * vis * wl.idx_heads * wl.idx_dim)}
+    g["topk_select"] = {"bytes": scores + sel, "flops": 0}
+    g["sparse_attn"] = {"bytes": rows + q + out + sel + H * 4,
+                        "flops": int(4 * n_q * H * n_rows * d)}
+    # the step's own bytes: scores and indices stay between its kernels
+    g["step"] = {"bytes": sum(v["bytes"] for v in g.values()) - 2 * scores - 2 * sel}
+    return g
 
 
 # ------------------------------------------------------------------ clocks
@@ -176,54 +201,7 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm), "source": "nvml, 20 ms"}
 
 
-# ------------------------------------------------------------------ reference arm
-def run_reference(args, rank):
-    if rank != 0:
-        return 0
-    import numpy as np
-    import oracle
-    from sparse_compressed_attention_csa_b200 import workloads as W
-    wl = _workload()
-    one = wl.replace(B=1)  # sequence 0 of the workload: the generator's streams are per tensor
-    data = W.generate(one)
-    f = W.to_f64
-
-    def step():
-        qp = data["q_pos"][0]
-        idx = oracle.index_topk(f(data["q_idx"][0]), data["w"][0], f(data["k_idx"][0]), qp,
-                                int(data["n_cmp"][0]), wl.width, wl.stride, wl.topk)
-        return oracle.sparse_attn(f(data["q"][0]), qp, W.bits_to_f32(data["kv_cmp"][0]), idx,
-                                  W.bits_to_f32(data["kv_raw"][0]), int(data["raw_pos0"][0]),
-                                  int(data["n_raw"][0]), data["sink"], wl.scale, wl.window,
-                                  wl.rope_dim, wl.theta)
-
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    step()
-    t_one = time.perf_counter() - t0
-    budget = 150.0
-    steps = args.steps if t_one * args.steps <= budget else max(3, int(budget / t_one))
-    t0 = time.perf_counter()
-    for _ in range(steps):
-        step()
-    el = time.perf_counter() - t0
-    value = steps * wl.n_heads / el
-    cores = _blas_threads()
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * el / steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": _config(wl),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": "one of the 32 sequences per step (its indexer, top-k and "
-                                       "128-head attention), fp64 NumPy oracle"},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
-                    "d2h_bytes_per_step": 0}}
-    print(json.dumps(line))
-    return 0
-
-
+# ------------------------------------------------------------------ oracle arm
 def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -235,31 +213,99 @@ def _blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, budget_s=12.0):
-    """The oracle on whole sequences of the workload, until ~budget_s elapsed."""
+def _oracle_sample(wl):
+    """(step function, query-heads per step, description): the fp64 oracle on
+    a bounded sample of the workload."""
+    import numpy as np
+
     import oracle
     from sparse_compressed_attention_csa_b200 import workloads as W
-    one = wl.replace(B=1)
-    data = W.generate(one)
     f = W.to_f64
-    t0 = time.perf_counter()
-    n = 0
-    while True:
+    v = W.bits_to_f32
+    if wl.kind == "csa_prefill":
+        data = W.generate(wl)
+        rows = np.linspace(0, wl.T - 1, 16).astype(np.int64)
+
+        def step():
+            kv = oracle.compress(f(data["x"][0]), f(data["g"][0]), wl.width, wl.stride,
+                                 wl.rope_dim, wl.theta, wl.pos_offset)
+            raw = oracle.rotate_raw(f(data["x"][0]), 0, wl.rope_dim, wl.theta)
+            qp = data["q_pos"][0]
+            idx = oracle.index_topk(v(data["q_idx"][0]), data["w"][0], f(data["k_idx"][0]), qp,
+                                    kv.shape[0], wl.width, wl.stride, wl.topk, rows)
+            return oracle.sparse_attn(f(data["q"][0][rows]), qp[rows], kv, idx, raw, 0, wl.T,
+                                      data["sink"], wl.scale, wl.window, wl.rope_dim, wl.theta)
+        return step, len(rows) * wl.n_heads, (
+            "compression of the whole sequence, then the indexer, top-k and 128-head attention "
+            "for 16 of the 8,192 query tokens, fp64 NumPy oracle")
+    one = wl.replace(B=1)  # sequence 0 of the workload: the generator's streams are per tensor
+    data = W.generate(one)
+    if wl.kind == "hca_decode":
+        def step():
+            return oracle.hca_attn(f(data["q"][0]), data["q_pos"][0], v(data["kv_cmp"][0]),
+                                   int(data["n_cmp"][0]), v(data["kv_raw"][0]),
+                                   int(data["raw_pos0"][0]), int(data["n_raw"][0]), data["sink"],
+                                   wl.scale, wl.window, wl.width, wl.stride, wl.rope_dim,
+                                   wl.theta)
+        return step, wl.n_heads, (f"one of the {wl.B} sequences per step (128-head attention "
+                                  f"over its {wl.n_cmp} entries and window), fp64 NumPy oracle")
+
+    def step():
         qp = data["q_pos"][0]
         idx = oracle.index_topk(f(data["q_idx"][0]), data["w"][0], f(data["k_idx"][0]), qp,
                                 int(data["n_cmp"][0]), wl.width, wl.stride, wl.topk)
-        oracle.sparse_attn(f(data["q"][0]), qp, W.bits_to_f32(data["kv_cmp"][0]), idx,
-                           W.bits_to_f32(data["kv_raw"][0]), int(data["raw_pos0"][0]),
-                           int(data["n_raw"][0]), data["sink"], wl.scale, wl.window, wl.rope_dim,
-                           wl.theta)
+        return oracle.sparse_attn(f(data["q"][0]), qp, v(data["kv_cmp"][0]), idx,
+                                  v(data["kv_raw"][0]), int(data["raw_pos0"][0]),
+                                  int(data["n_raw"][0]), data["sink"], wl.scale, wl.window,
+                                  wl.rope_dim, wl.theta)
+    return step, wl.n_heads, (f"one of the {wl.B} sequences per step (indexer over "
+                              f"{wl.n_cmp:,} entries, top-{wl.topk}, 128-head attention), "
+                              f"fp64 NumPy oracle")
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    wl = _workload(args.workload, args.batch)
+    step, qh, desc = _oracle_sample(wl)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    step()
+    t_one = time.perf_counter() - t0
+    budget = 150.0
+    steps = args.steps if t_one * args.steps <= budget else max(3, int(budget / t_one))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    el = time.perf_counter() - t0
+    value = steps * qh / el
+    line = {"impl": "reference", "metric": _metric(wl), "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": steps, "steps_requested": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * el / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    """The oracle on the sample of `_oracle_sample`, until ~budget_s elapsed."""
+    step, qh, desc = _oracle_sample(wl)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        step()
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 64:
             break
-    return {"value": n * wl.n_heads / el, "unit": UNIT, "cores": _blas_threads(),
-            "kind": "oracle",
-            "sample": f"{n} whole sequence(s) of the workload (indexer over 16,383 entries, "
-                      f"top-1024, 128-head attention), fp64 NumPy, {el:.1f} s"}
+    return {"value": n * qh / el, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{n} step(s) of: {desc}; {el:.1f} s"}
 
 
 # ------------------------------------------------------------------ CUDA arm
@@ -280,7 +326,7 @@ def run_cuda(args, rank, world, local):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    wl = _workload()
+    wl = _workload(args.workload, args.batch)
     data = W.generate(wl)
 
     def todev(a):
@@ -289,32 +335,60 @@ def run_cuda(args, rank, world, local):
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
     t = {k: todev(v) for k, v in data.items()}
-    p = L.Params(topk=wl.topk, window=wl.window)
-    Bsz, Tq, N = wl.B, 1, wl.n_cmp
-    scores = torch.empty((Bsz, Tq, N), dtype=torch.float32, device=dev)
-    idx = torch.empty((Bsz, Tq, wl.topk), dtype=torch.int32, device=dev)
+    p = L.Params(d=wl.d, rope_dim=wl.rope_dim, theta=wl.theta, scale=wl.scale,
+                 n_heads=wl.n_heads, idx_heads=wl.idx_heads, idx_dim=wl.idx_dim, topk=wl.topk,
+                 window=wl.window, width=wl.width, stride=wl.stride, pos_offset=wl.pos_offset)
+    Bsz, Tq, N = wl.B, wl.Tq, wl.n_cmp
     out = torch.empty_like(t["q"])
-    ws_topk = L.csa_workspace_size(p, L.CSA_OP_TOPK_SELECT, Bsz, Tq, N)
-    ws_attn = L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, Bsz, Tq, N)
-    ws = torch.empty(max(ws_topk, ws_attn, 256), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)  # 256 MiB
+    ops = {"hca_decode": [L.CSA_OP_HCA_ATTN]}.get(
+        wl.kind, [L.CSA_OP_TOPK_SELECT, L.CSA_OP_SPARSE_ATTN])
+    ws = torch.empty(max([L.csa_workspace_size(p, o, Bsz, Tq, N) for o in ops] + [256]),
+                     dtype=torch.uint8, device=dev)
+    if wl.kind != "hca_decode":
+        scores = torch.empty((Bsz, Tq, N), dtype=torch.float32, device=dev)
+        idx = torch.empty((Bsz, Tq, wl.topk), dtype=torch.int32, device=dev)
+    if wl.kind == "csa_prefill":
+        t["kv_cmp"] = torch.empty((Bsz, N, wl.d), dtype=torch.bfloat16, device=dev)
+        t["kv_raw"] = torch.empty((Bsz, wl.T, wl.d), dtype=torch.bfloat16, device=dev)
+
+    # the step's kernel groups, in order
+    groups = []
+    if wl.kind == "csa_prefill":
+        groups.append(("compress", lambda: L.csa_compress(p, t["x"], t["g"], t["kv_cmp"],
+                                                          t["kv_raw"])))
+    if wl.kind == "hca_decode":
+        groups.append(("hca_attn", lambda: L.hca_attn(
+            p, t["q"], t["q_pos"], t["kv_cmp"], t["n_cmp"], t["kv_raw"], t["raw_pos0"],
+            t["n_raw"], t["sink"], out, ws)))
+    else:
+        groups.append(("index_scores", lambda: L.csa_index_scores(
+            p, t["q_idx"], t["w"], t["k_idx"], t["q_pos"], t["n_cmp"], scores)))
+        groups.append(("topk_select", lambda: L.csa_topk_select(
+            p, scores, t["q_pos"], t["n_cmp"], idx, ws)))
+        groups.append(("sparse_attn", lambda: L.csa_sparse_attn(
+            p, t["q"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"], t["n_raw"],
+            t["sink"], out, ws)))
+
+    mib = max(args.flush_mib, 0)
+    flush = torch.empty(mib << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(mib << 18, dtype=torch.float32, device=dev)
 
     def flush_l2():
-        flush.zero_()
-        flush_rd.sum()  # evicts the dirty lines of the write: L2 left clean
+        if mib:
+            flush.zero_()
+            flush_rd.sum()  # evicts the dirty lines of the write: L2 left clean
     stream = torch.cuda.Stream(device=dev)
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(groups) + 1)]
 
-    def launch():
-        ev[0].record()
-        L.csa_index_scores(p, t["q_idx"], t["w"], t["k_idx"], t["q_pos"], t["n_cmp"], scores)
-        ev[1].record()
-        L.csa_topk_select(p, scores, t["q_pos"], t["n_cmp"], idx, ws)
-        ev[2].record()
-        L.csa_sparse_attn(p, t["q"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"],
-                          t["n_raw"], t["sink"], out, ws)
-        ev[3].record()
+    def launch(marks=False):
+        # marks: events between the kernels, for the per-kernel breakdown
+        # (they cut the programmatic-launch overlap, so the timed step has none)
+        for i, (_, fn) in enumerate(groups):
+            if marks:
+                ev[i].record()
+            fn()
+        if marks:
+            ev[len(groups)].record()
 
     with torch.cuda.stream(stream):
         n0 = L.csa_launch_count()
@@ -325,22 +399,35 @@ def run_cuda(args, rank, world, local):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         launch()
+    graph_marked = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_marked, stream=stream):
+        launch(marks=True)
     torch.cuda.synchronize()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
 
     def timed_steps(n):
-        tot = [0.0, 0.0, 0.0, 0.0]
+        tot = 0.0
         for _ in range(n):
             with torch.cuda.stream(stream):
                 flush_l2()
+                s0.record()
                 graph.replay()
+                s1.record()
             stream.synchronize()
-            a, b, c = (ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
-                       ev[2].elapsed_time(ev[3]))
-            tot[0] += a + b + c
-            tot[1] += a
-            tot[2] += b
-            tot[3] += c
+            tot += s0.elapsed_time(s1)
         return tot
+
+    def breakdown(n):
+        tot = [0.0] * len(groups)
+        for _ in range(n):
+            with torch.cuda.stream(stream):
+                flush_l2()
+                graph_marked.replay()
+            stream.synchronize()
+            for i in range(len(groups)):
+                tot[i] += ev[i].elapsed_time(ev[i + 1])
+        return [x / n for x in tot]
 
     timed_steps(args.warmup)
     sampler = ClockSampler(dev) if not args.no_clocks else None
@@ -356,18 +443,22 @@ def run_cuda(args, rank, world, local):
     clocks = sampler.stop() if sampler else None
     L.csa_poll_device_error(stream)
 
-    step_ms = tot[0] / args.steps
+    step_ms = tot / args.steps
+    n_bd = min(args.steps, 200)
+    bd = breakdown(n_bd)
     t_max = torch.tensor([step_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
     step_ms_max = float(t_max.item())
-    qh_per_step = wl.B * wl.n_heads
+    qh_per_step = wl.B * wl.Tq * wl.n_heads
     value = world * qh_per_step / (step_ms_max * 1e-3)
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host
+    h2d_keys = {"csa_decode": ("q", "q_idx", "w", "q_pos"), "hca_decode": ("q", "q_pos"),
+                "csa_prefill": ("x", "g", "q_idx", "w", "q")}[wl.kind]
     h_in = {k: torch.from_numpy(np.ascontiguousarray(data[k].view(np.int16) if data[k].dtype ==
                                                       np.uint16 else data[k])).pin_memory()
-            for k in ("q", "q_idx", "w", "q_pos")}
+            for k in h2d_keys}
     d_in = {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=dev) for k in h_in}
     h_out = torch.empty(out.shape, dtype=torch.int16).pin_memory()
     lw = layer.Workspace(dev)
@@ -376,32 +467,44 @@ def run_cuda(args, rank, world, local):
     h2d = sum(h_in[k].numel() * h_in[k].element_size() for k in h_in)
     d2h = h_out.numel() * h_out.element_size()
 
+    def bf(k):
+        return d_in[k].view(torch.bfloat16)
+
     def e2e_step():
         with torch.cuda.stream(stream):
             flush_l2()
             e_start.record()
             for k in h_in:
                 d_in[k].copy_(h_in[k], non_blocking=True)
-            q = d_in["q"].view(torch.bfloat16)
-            qi = d_in["q_idx"].view(torch.bfloat16)
-            _, o = layer.csa_decode(p, q, d_in["q_pos"], qi, d_in["w"], t["k_idx"], t["n_cmp"],
-                                    t["kv_cmp"], t["kv_raw"], t["raw_pos0"], t["n_raw"],
-                                    t["sink"], lw, idx=idx, out=out)
+            if wl.kind == "csa_decode":
+                _, o = layer.csa_decode(p, bf("q"), d_in["q_pos"], bf("q_idx"), d_in["w"],
+                                        t["k_idx"], t["n_cmp"], t["kv_cmp"], t["kv_raw"],
+                                        t["raw_pos0"], t["n_raw"], t["sink"], lw, idx=idx,
+                                        out=out)
+            elif wl.kind == "hca_decode":
+                o = layer.hca_decode(p, bf("q"), d_in["q_pos"], t["kv_cmp"], t["n_cmp"],
+                                     t["kv_raw"], t["raw_pos0"], t["n_raw"], t["sink"], lw,
+                                     out=out)
+            else:
+                _, _, _, o = layer.csa_prefill(p, bf("x"), bf("g"), bf("q_idx"), d_in["w"],
+                                               t["k_idx"], bf("q"), t["sink"], lw)
             h_out.copy_(o.view(torch.int16), non_blocking=True)
             e_end.record()
         stream.synchronize()
         return e_start.elapsed_time(e_end)
 
+    n_e2e = min(args.steps, 100)
     for _ in range(args.warmup):
         e2e_step()
     if world > 1:
         dist.barrier()
-    e2e_ms = sum(e2e_step() for _ in range(args.steps)) / args.steps
+    e2e_ms = sum(e2e_step() for _ in range(n_e2e)) / n_e2e
     e_max = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(e_max, op=dist.ReduceOp.MAX)
         dist.barrier()
     e2e_value = world * qh_per_step / (float(e_max.item()) * 1e-3)
+    L.csa_poll_device_error(stream)
 
     if rank == 0:
         peaks = {}
@@ -411,32 +514,32 @@ def run_cuda(args, rank, world, local):
         hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
         tc = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
         work = algorithmic_work(wl)
-        kernel_ms = {"index_scores": tot[1] / args.steps, "topk_select": tot[2] / args.steps,
-                     "sparse_attn": tot[3] / args.steps}
-        traffic = _recorded_traffic(wl)
+        kernel_ms = {name: bd[i] for i, (name, _) in enumerate(groups)}
         rl = {}
         for k, ms in kernel_ms.items():
             b, f = work[k]["bytes"], work[k]["flops"]
             gbs = b / (ms * 1e-3) / 1e9
             tfl = f / (ms * 1e-3) / 1e12
-            # the bound is the roof the kernel's arithmetic intensity meets first
+            # the bound is the roof that the kernel's arithmetic intensity meets first
             tensor = f > 0 and f / b > tc * 1e12 / (hbm * 1e9)
             rl[k] = {"bound": "tensor" if tensor else "hbm",
                      "achieved": tfl if tensor else gbs, "peak": tc if tensor else hbm,
                      "unit": "TFLOP/s" if tensor else "GB/s",
                      "frac": (tfl / tc) if tensor else (gbs / hbm),
                      "algorithmic_bytes": b, "flops": f, "ms": ms,
-                     "tensor_frac": tfl / tc if f else 0.0,
-                     "traffic": traffic.get(k), "peak_source": src + " burst"}
+                     "hbm_frac": gbs / hbm, "tensor_frac": tfl / tc if f else 0.0,
+                     "traffic": None, "peak_source": src + " burst"}
         dom = max(kernel_ms, key=kernel_ms.get)
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "metric": _metric(wl), "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": _config(wl),
+            "data": "synthetic", "config": _config(wl, flush_mib=mib),
             "gpu_launches": kernels_per_step * args.steps,
             "kernels_per_step": kernels_per_step,
             "kernel_ms": kernel_ms,
+            "kernel_ms_note": f"{n_bd} steps of the same graph with events between the launches "
+                              "(no programmatic-launch overlap there); the timed step has none",
             "step_hbm": {"algorithmic_bytes": work["step"]["bytes"],
                          "achieved_gbs": work["step"]["bytes"] / (step_ms_max * 1e-3) / 1e9,
                          "frac": work["step"]["bytes"] / (step_ms_max * 1e-3) / 1e9 / hbm,
@@ -446,13 +549,13 @@ def run_cuda(args, rank, world, local):
                                                      "traffic", "peak_source")}),
             "roofline_by_kernel": rl,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "steps": n_e2e},
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl)
         print(json.dumps(line))
-    del graph
+    del graph, graph_marked
     if world > 1:
         dist.destroy_process_group()
     return 0

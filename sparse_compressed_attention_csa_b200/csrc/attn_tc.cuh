@@ -34,8 +34,13 @@
 //   warps 0-3: one head per thread (= TMEM lane): online softmax in the
 //              log2 domain with a lazy rescale (only when the running max
 //              grows by more than 2^8), P written back over S as bf16,
-//              epilogue with the sink, the inverse output rotation and the
-//              store (or split-KV partials for k_attn_combine).
+//              epilogue with the sink, the inverse output rotation and a
+//              TMA store of the bf16 output.
+//
+// Split-KV (few query tokens): the S splits of one (token, part) form a
+// thread-block cluster.  Each writes its (m, l) and partial O to the
+// workspace; after a cluster barrier each CTA merges 1/S of the output dims
+// over all splits.
 // Every mbarrier wait is bounded; a timeout records CSA_ERR_DEVICE_TIMEOUT
 // and the CTA winds down, frees TMEM and exits.
 #pragma once
@@ -52,7 +57,9 @@ constexpr int kAtSubBytes = kAtHeads * 128;       // q box: [128 heads][64 dims]
 constexpr int kAtRowCap = 2048;                   // rows per query token
 constexpr int kAtMaxRope = 128;                   // rotated dims supported
 constexpr int kAtMaxSlots = 13;
-constexpr int kAtMaxSplits = 16;                  // split-KV parts per query token
+constexpr int kAtMaxSplits = 8;                   // split-KV parts per query token (one cluster)
+constexpr int kAtSlabBytes = kAtHeads * 32 * 4;    // 32 dims of fp32 O for 128 heads
+constexpr int kAtOutBoxBytes = kAtHeads * 64;      // 32 dims of bf16 output for 128 heads
 constexpr int kAtThreads = 288;
 constexpr float kAtRescaleLog2 = 8.0f;
 
@@ -72,9 +79,8 @@ struct AttnTcArgs {
   float scale_log2;
   int splits;
   __nv_bfloat16* out;  // splits == 1
-  float* part_o;       // splits > 1: [B*Tq][splits][NQ][512/NQ/32][8][128][4]
-  float* part_ml;      // [B*Tq][splits][NQ][2][128]  (m, l)
-  int* arrive;         // [B*Tq][NQ] split arrivals, zero before the launch
+  float* part_o;       // splits > 1: [B*Tq][NQ][splits][512/NQ/32 slabs][8][128][4]
+  float* part_ml;      // [B*Tq][NQ][splits][2][128]  (m, l)
   double freq[kAtMaxRope / 2];  // RoPE frequencies theta^(-2i/rope_dim)
 };
 
@@ -104,6 +110,20 @@ struct AtLayout {
   static constexpr uint32_t kTmemS = kOCols;         // S0, S1: 2 x 64 columns
   static constexpr uint32_t kTmemQ = kOCols + 128;   // Q chunks held in TMEM
 };
+// Idle shared memory the epilogue needs with S splits: (S - 1) partial slabs
+// of the merged range per other split, plus the output boxes.
+template <int NQ>
+constexpr int at_epilogue_bytes() {
+  int worst = (kAtDim / NQ / 32) * kAtOutBoxBytes;  // S = 1: every slab
+  for (int S = 2; S <= kAtMaxSplits; ++S) {
+    const int ns = (kAtDim / NQ / 32 + S - 1) / S;
+    const int need = (S - 1) * ns * kAtSlabBytes + ns * kAtOutBoxBytes;
+    worst = need > worst ? need : worst;
+  }
+  return worst;
+}
+static_assert(at_epilogue_bytes<2>() <= AtLayout<2>::kMiscOff, "epilogue buffers (NQ = 2)");
+static_assert(at_epilogue_bytes<4>() <= AtLayout<4>::kMiscOff, "epilogue buffers (NQ = 4)");
 static_assert(AtLayout<2>::kBytes + 1024 <= 232448, "shared memory budget (NQ = 2)");
 static_assert(AtLayout<4>::kBytes + 1024 <= 232448, "shared memory budget (NQ = 4)");
 
@@ -145,6 +165,12 @@ __device__ __forceinline__ uint32_t swz(int r, int u) {
   return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4));
 }
 
+// Byte offset of 16-byte unit u (0..3) of row r inside a 64B-swizzled
+// [rows][64 B] block (the 16-byte unit index XOR bits 1-2 of the row).
+__device__ __forceinline__ uint32_t swz64(int r, int u) {
+  return (uint32_t)(r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
+}
+
 // cos / sin of pos * freq: the angle is reduced modulo 2 pi in double
 // precision (2 pi split in two parts), then taken in fp32.
 __device__ __forceinline__ void rope_cs_reduced(long long pos, double freq, float* c, float* s) {
@@ -171,12 +197,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint8_t* ring = base_ptr + Lay::kRingOff;  // kSlots x 16 KB
   AtMisc& sm = *reinterpret_cast<AtMisc*>(base_ptr + Lay::kMiscOff);
 
-  const int part = blockIdx.x % NQ;
-  const int split = blockIdx.x / NQ;
+  // the splits of one (token, part) are consecutive in x: one cluster
+  const int S = a.splits;
+  const int split = blockIdx.x % S;
+  const int part = blockIdx.x / S;
   const int row_q = blockIdx.y;  // b * Tq + tq
   const int b = row_q / a.Tq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = a.q_pos[row_q];
   const int rope0 = kAtDim - a.rope_dim;
   // 128-dim chunks in streaming order: the others first, then the own ones
   // (own chunks: dims part * kOCols ..)
@@ -223,6 +250,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const uint32_t t_o = tmem, t_s = tmem + Lay::kTmemS, t_q = tmem + Lay::kTmemQ;
   volatile int* abortp = &sm.abort_flag;
+  griddep_wait();  // the predecessor's writes (the selected indices) are visible
+  griddep_launch_dependents();
+  const int t = a.q_pos[row_q];
 
   if (warp == 4 && lane == 0) {
     // q of this token: 8 boxes of [128 heads][64 dims], 128B swizzle
@@ -333,6 +363,57 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     ntile = (nrow + kAtTile - 1) / kAtTile;
   };
 
+  // Epilogue helpers (warps 0-3, one head per thread).  The output leaves
+  // as 32-dim slabs: bf16 TMA boxes of [128 heads][64 B], 64B-swizzled,
+  // staged in shared memory that is idle by then.
+  float m_run = -INFINITY, l_run = 0.f;  // this split's softmax state of the thread's head
+  bool epi_ok = false;
+  auto out_slab = [&](uint8_t* obuf, int sl, int box, float (&o)[32]) {
+    const int hd = threadIdx.x;
+    const int d0 = part * kOCols + sl * 32;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const int d = d0 + e;
+      if (d >= rope0) {  // inverse rotation at -t
+        const int ii = (d - rope0) >> 1;
+        const float x0 = o[e], x1 = o[e + 1];
+        o[e] = x0 * sm.cs[ii] + x1 * sm.sn[ii];
+        o[e + 1] = -x0 * sm.sn[ii] + x1 * sm.cs[ii];
+      }
+    }
+    uint8_t* bx = obuf + box * kAtOutBoxBytes;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<uint4*>(bx + swz64(hd, u)) =
+          make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]), pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
+                     pack_bf16x2(o[8 * u + 4], o[8 * u + 5]), pack_bf16x2(o[8 * u + 6], o[8 * u + 7]));
+  };
+  auto store_out = [&](uint8_t* obuf, int sl0, int n) {
+    fence_proxy_async_shared();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < n; ++i)
+        tma_store_2d(&tm_out, obuf + i * kAtOutBoxBytes, part * kOCols + (sl0 + i) * 32,
+                     row_q * kAtHeads);
+      bulk_commit();
+      bulk_wait_read_all();
+    }
+  };
+  // this CTA's O, slab sl, times w (zero without tiles)
+  auto own_slab = [&](int sl, uint32_t lane_base, float w, float (&o)[32]) {
+    uint32_t r[32];
+    if (ntile > 0) {
+      tmem_ld32(t_o + lane_base + (uint32_t)(sl * 32), r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __fmul_rn(__uint_as_float(r[e]), w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0.f;
+    }
+  };
+  constexpr int kSlabs = kOCols / 32;
+
   if (warp < 4) {
     // ======================= softmax / epilogue warps
     const int head = warp * 32 + lane;  // TMEM lane
@@ -396,7 +477,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
     // ---- online softmax over the tiles
     const int n_sel = sm.n_sel, ps = (n_sel + 3) & ~3, pe = ps + sm.n_win;
-    float m_run = -INFINITY, l_run = 0.f;
     for (int i = 0; i < ntile && ok; ++i) {
       const int sb = i & 1;
       const uint32_t ph = (uint32_t)(i >> 1) & 1u;
@@ -485,228 +565,44 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      // Shared memory is idle once the last PV has landed (q's own half and
-      // the ring are one contiguous block).  It holds, for a split-KV merge,
-      // one other split's partial O (pbuf, in its global layout) and, for
-      // the output, the bf16 tile of this CTA's dims as kOCols / 64 TMA boxes
-      // of [128 heads][128 B], 128B-swizzled.
-      constexpr int kPartBytes = kAtHeads * kOCols * 4;
-      constexpr int kOutBoxes = kOCols / 64;
-      static_assert(kPartBytes + kOutBoxes * kAtSubBytes + 2 * kAtMaxSplits * kAtHeads * 4 <=
-                        Lay::kMiscOff,
-                    "epilogue buffers exceed the idle shared memory");
-      uint8_t* pbuf = base_ptr;
-      uint8_t* obuf = base_ptr + kPartBytes;
-      const float sink_l2 = a.sink[head] * 1.4426950408889634f;
-      const int S = a.splits;
-      const size_t unit0 = (size_t)row_q * S * NQ + part;  // unit of split s: unit0 + s * NQ
-      // Partial O layout per unit: [slab of 32 dims][16-byte unit u][head][4
-      // floats], so that a warp's 16-byte accesses at one (slab, u) are
-      // contiguous.
-      auto part_off = [&](int cc, int u) { return ((size_t)((cc / 32) * 8 + u) * kAtHeads + head) * 4; };
-      // One pass over the 32-column slabs.  Terms src * w, in split order:
-      // this CTA's O (TMEM; zero without tiles) and/or the partial in pbuf
-      // (`buf_first`: the pbuf term comes first).  acc = terms (`first`) or
-      // acc + terms, the running sum kept in TMEM columns [t_s, t_s +
-      // kOCols) (S and q are dead by now).  mode 0: acc back to TMEM; 1: out
-      // as this split's fp32 partial; 2: rotated back at -t, rounded to bf16
-      // and stored through TMA.  Every product and sum is rounded on its own,
-      // in split order, so a merge does not depend on which split performs
-      // it.
-      const uint32_t t_acc = t_s;
-      auto slab_pass = [&](bool use_own, float w_own, bool use_buf, float w_buf, bool buf_first,
-                           bool first, int mode) {
-#pragma unroll 1
-        for (int cc = 0; cc < kOCols; cc += 32) {
-          float o[32];
-          bool have = !first;
-          if (have) {
-            uint32_t r[32];
-            tmem_ld32(t_acc + lane_base + (uint32_t)cc, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(r[e]);
-          }
-          auto add_own = [&]() {
-            uint32_t r[32];
-            if (ntile > 0) {
-              tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
-              tmem_wait_ld();
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = 0u;
-            }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float tm = __fmul_rn(__uint_as_float(r[e]), w_own);
-              o[e] = have ? __fadd_rn(o[e], tm) : tm;
-            }
-            have = true;
-          };
-          auto add_buf = [&]() {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float4 x =
-                  *reinterpret_cast<const float4*>(pbuf + part_off(cc, u) * sizeof(float));
-              const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const float tm = __fmul_rn(xs[v], w_buf);
-                o[4 * u + v] = have ? __fadd_rn(o[4 * u + v], tm) : tm;
-              }
-            }
-            have = true;
-          };
-          if (use_buf && buf_first) add_buf();
-          if (use_own) add_own();
-          if (use_buf && !buf_first) add_buf();
-          if (mode == 0) {
-            uint32_t w16[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(o[e]);
-            tmem_st16(t_acc + lane_base + (uint32_t)cc, w16);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(o[16 + e]);
-            tmem_st16(t_acc + lane_base + (uint32_t)cc + 16, w16);
-          } else if (mode == 1) {
-            float* dst = a.part_o + (unit0 + (size_t)split * NQ) * kAtHeads * kOCols;
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<float4*>(dst + part_off(cc, u)) =
-                  make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
-          } else {
-            const int d0 = part * kOCols + cc;
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int d = d0 + e;
-              if (d >= rope0) {  // inverse rotation at -t
-                const int ii = (d - rope0) >> 1;
-                const float x0 = o[e], x1 = o[e + 1];
-                o[e] = x0 * sm.cs[ii] + x1 * sm.sn[ii];
-                o[e + 1] = -x0 * sm.sn[ii] + x1 * sm.cs[ii];
-              }
-            }
-            uint8_t* box = obuf + (cc / 64) * kAtSubBytes;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int u = ((cc & 63) >> 3) + j;
-              *reinterpret_cast<uint4*>(box + swz(head, u)) =
-                  make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
-                             pack_bf16x2(o[8 * j + 4], o[8 * j + 5]), pack_bf16x2(o[8 * j + 6], o[8 * j + 7]));
-            }
-          }
-        }
-        if (mode == 0) {
-          tmem_wait_st();
-          tc_fence_before();
-        } else if (mode == 2) {
-          fence_proxy_async_shared();
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (threadIdx.x == 0) {
-            for (int bx = 0; bx < kOutBoxes; ++bx)
-              tma_store_2d(&tm_out, obuf + bx * kAtSubBytes, part * kOCols + bx * 64,
-                           row_q * kAtHeads);
-            bulk_commit();
-            bulk_wait_read_all();
-          }
-        }
-      };
       if (S == 1) {
+        // shared memory is idle once the last PV has landed
+        const float sink_l2 = a.sink[head] * 1.4426950408889634f;
         const float mm = fmaxf(m_run, sink_l2);
         const float den = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - mm)) +
                           exp2f(sink_l2 - mm);
         const float scl =
             (m_run == -INFINITY || !(den > 0.f)) ? 0.f : exp2f(m_run - mm) / den;
-        slab_pass(true, scl, false, 0.f, false, true, 2);
+#pragma unroll 1
+        for (int sl = 0; sl < kSlabs; ++sl) {
+          float o[32];
+          own_slab(sl, lane_base, scl, o);
+          out_slab(base_ptr, sl, sl, o);
+        }
+        store_out(base_ptr, 0, kSlabs);
       } else {
-        // split-KV: publish (m, l, O) of this split; the last split of the
-        // (token, part) to finish merges all of them in split order (its
-        // own O straight from TMEM) and resets the arrival counter
-        float* pml = a.part_ml + (unit0 + (size_t)split * NQ) * 2 * kAtHeads;
+        // split-KV: publish this split's (m, l) and the slabs of O that the
+        // other splits of the cluster merge (layout per unit: [slab][16-byte
+        // unit u][head][4 floats], so that a warp's stores coalesce)
+        const size_t unit = ((size_t)row_q * NQ + part) * S + split;
+        float* pml = a.part_ml + unit * 2 * kAtHeads;
         pml[head] = m_run;
         pml[kAtHeads + head] = l_run;
-        slab_pass(true, 1.f, false, 0.f, false, true, 1);
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (threadIdx.x == 0) {
-          const int old = atomicAdd(a.arrive + (size_t)row_q * NQ + part, 1);
-          sm.scan_tmp[0] = old == S - 1 ? 1 : 0;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (sm.scan_tmp[0]) {
-          __threadfence();
-          fence_proxy_async_global();  // the partials are read by bulk copies
-          // (m, l) of every split for this thread's head, in one batch of loads
-          float* mls = reinterpret_cast<float*>(obuf + kOutBoxes * kAtSubBytes);
-#pragma unroll 4
-          for (int sp = 0; sp < S; ++sp) {
-            const float* ml = a.part_ml + (unit0 + (size_t)sp * NQ) * 2 * kAtHeads;
-            mls[(2 * sp) * kAtHeads + head] = sp == split ? m_run : __ldcg(ml + head);
-            mls[(2 * sp + 1) * kAtHeads + head] = sp == split ? l_run : __ldcg(ml + kAtHeads + head);
-          }
-          float M = sink_l2;
-          for (int sp = 0; sp < S; ++sp) M = fmaxf(M, mls[(2 * sp) * kAtHeads + head]);
-          float L = exp2f(sink_l2 - M);
-          for (int sp = 0; sp < S; ++sp) {
-            const float m = mls[(2 * sp) * kAtHeads + head];
-            if (m != -INFINITY) L += mls[(2 * sp + 1) * kAtHeads + head] * exp2f(m - M);
-          }
-          const float inv = L > 0.f ? 1.f / L : 0.f;
-          auto weight = [&](int sp) {
-            const float m = mls[(2 * sp) * kAtHeads + head];
-            return m == -INFINITY ? 0.f : exp2f(m - M) * inv;
-          };
-          int loads = 0;
-          bool okm = true;
-          auto fetch = [&](int sp) -> bool {  // partial O of split sp into pbuf
-            if (threadIdx.x == 0) {
-              mbar_arrive_expect_tx(&sm.merge_bar, kPartBytes);
-              bulk_load(pbuf, a.part_o + (unit0 + (size_t)sp * NQ) * kAtHeads * kOCols,
-                        kPartBytes, &sm.merge_bar);
-            }
-            bool got = __all_sync(0xffffffffu,
-                                  mbar_wait(&sm.merge_bar, (uint32_t)(loads & 1), abortp));
-            ++loads;
-            uint32_t all;  // the four warps agree before going on
-            asm volatile(
-                "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-                "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                : "=r"(all)
-                : "r"(got ? 1u : 0u)
-                : "memory");
-            return all != 0;
-          };
-          // passes over the splits in order; this CTA's own O joins the pass
-          // of its neighbour, so two splits take one pass and one copy
-          bool first = true;
-          for (int sp = 0; sp < S && okm;) {
-            if (sp == split) {
-              if (sp + 1 < S) {
-                okm = fetch(sp + 1);
-                if (!okm) break;
-                slab_pass(true, weight(sp), true, weight(sp + 1), false, first,
-                          sp + 2 == S ? 2 : 0);
-                sp += 2;
-              } else {
-                slab_pass(true, weight(sp), false, 0.f, false, first, 2);
-                sp += 1;
-              }
-            } else {
-              okm = fetch(sp);
-              if (!okm) break;
-              const bool with_own = sp + 1 == split;
-              const int next = sp + (with_own ? 2 : 1);
-              slab_pass(with_own, with_own ? weight(sp + 1) : 0.f, true, weight(sp), true, first,
-                        next == S ? 2 : 0);
-              sp = next;
-            }
-            first = false;
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // pbuf free again
-          }
-          if (threadIdx.x == 0) a.arrive[(size_t)row_q * NQ + part] = 0;
+        float* dst = a.part_o + unit * kAtHeads * kOCols;
+        const int my_lo = split * kSlabs / S, my_hi = (split + 1) * kSlabs / S;
+#pragma unroll 1
+        for (int sl = 0; sl < kSlabs; ++sl) {
+          if (sl >= my_lo && sl < my_hi) continue;
+          float o[32];
+          own_slab(sl, lane_base, 1.f, o);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(dst + ((size_t)(sl * 8 + u) * kAtHeads + head) * 4) =
+                make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         }
       }
     }
+    epi_ok = ok;
   } else if (warp < 8) {
     // ======================= gather producers (128 threads)
     // Chunk n (tile n / 4, part n % 4 in streaming order) goes to ring slot
@@ -841,6 +737,103 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       mbar_wait(&sm.s_full[last_s & 1], (uint32_t)(last_s >> 1) & 1u, &never, 100000000ull);
     if (last_pv >= 0)
       mbar_wait(&sm.pv_done[last_pv & 1], (uint32_t)(last_pv >> 1) & 1u, &never, 100000000ull);
+  }
+  if (S > 1) {
+    // ======================= split-KV merge inside the cluster: after the
+    // barrier every split's (m, l) and partial O are visible; CTA `split`
+    // merges output slabs [split * kSlabs / S, (split + 1) * kSlabs / S) in
+    // split order (its own O straight from TMEM, the others' from a bulk
+    // copy).  Products and sums are rounded one by one, in split order, so
+    // the result does not depend on the merging CTA.
+    __syncwarp();
+    cluster_sync_all();
+    if (warp < 4 && epi_ok) {
+      const int head = threadIdx.x;
+      const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+      const int s_lo = split * kSlabs / S, s_hi = (split + 1) * kSlabs / S, ns = s_hi - s_lo;
+      const size_t unit0 = ((size_t)row_q * NQ + part) * S;  // unit of split sp: unit0 + sp
+      uint8_t* pbuf = base_ptr;                           // (S - 1) x ns slabs of 16 KB
+      uint8_t* obuf = base_ptr + (S - 1) * ns * kAtSlabBytes;  // ns output boxes
+      bool okm = ns > 0;
+      if (okm && threadIdx.x == 0) {
+        fence_proxy_async_global();  // partials written by generic stores, read by bulk copies
+        mbar_arrive_expect_tx(&sm.merge_bar, (uint32_t)((S - 1) * ns * kAtSlabBytes));
+        for (int sp = 0, j = 0; sp < S; ++sp) {
+          if (sp == split) continue;
+          bulk_load(pbuf + j * ns * kAtSlabBytes,
+                    a.part_o + (unit0 + sp) * kAtHeads * kOCols + (size_t)s_lo * (kAtSlabBytes / 4),
+                    (uint32_t)(ns * kAtSlabBytes), &sm.merge_bar);
+          ++j;
+        }
+      }
+      // merge weights of the thread's head: exp(m_s - M) / L with the sink
+      const float sink_l2 = a.sink[head] * 1.4426950408889634f;
+      float mv[kAtMaxSplits], lv[kAtMaxSplits];
+#pragma unroll
+      for (int sp = 0; sp < kAtMaxSplits; ++sp) {
+        mv[sp] = -INFINITY;
+        lv[sp] = 0.f;
+        if (sp < S) {
+          const float* ml = a.part_ml + (unit0 + sp) * 2 * kAtHeads;
+          mv[sp] = sp == split ? m_run : __ldcg(ml + head);
+          lv[sp] = sp == split ? l_run : __ldcg(ml + kAtHeads + head);
+        }
+      }
+      float M = sink_l2;
+#pragma unroll
+      for (int sp = 0; sp < kAtMaxSplits; ++sp) M = fmaxf(M, mv[sp]);
+      float L = exp2f(sink_l2 - M);
+#pragma unroll
+      for (int sp = 0; sp < kAtMaxSplits; ++sp)
+        if (mv[sp] != -INFINITY) L += lv[sp] * exp2f(mv[sp] - M);
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+      for (int sp = 0; sp < kAtMaxSplits; ++sp)
+        mv[sp] = mv[sp] == -INFINITY ? 0.f : exp2f(mv[sp] - M) * inv;  // now the weights
+      if (okm) okm = __all_sync(0xffffffffu, mbar_wait(&sm.merge_bar, 0, abortp));
+      {  // the four warps agree before the named barrier of store_out
+        uint32_t all;
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+            "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(all)
+            : "r"(okm ? 1u : 0u)
+            : "memory");
+        okm = all != 0;
+      }
+      if (okm) {
+#pragma unroll 1
+        for (int sl = s_lo; sl < s_hi; ++sl) {
+          float o[32];
+          bool have = false;
+          int j = 0;
+#pragma unroll
+          for (int sp = 0; sp < kAtMaxSplits; ++sp) {
+            if (sp >= S) break;
+            float tm[32];
+            if (sp == split) {
+              own_slab(sl, lane_base, mv[sp], tm);
+            } else {
+              const uint8_t* src = pbuf + (j * ns + (sl - s_lo)) * kAtSlabBytes;
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const float4 x = *reinterpret_cast<const float4*>(src + (u * kAtHeads + head) * 16);
+                tm[4 * u] = __fmul_rn(x.x, mv[sp]);
+                tm[4 * u + 1] = __fmul_rn(x.y, mv[sp]);
+                tm[4 * u + 2] = __fmul_rn(x.z, mv[sp]);
+                tm[4 * u + 3] = __fmul_rn(x.w, mv[sp]);
+              }
+              ++j;
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = have ? __fadd_rn(o[e], tm[e]) : tm[e];
+            have = true;
+          }
+          out_slab(obuf, sl, sl - s_lo, o);
+        }
+        store_out(obuf, s_lo, ns);
+      }
+    }
   }
   // every copy issued into shared memory has landed before the CTA may exit
   if (warp == 4 && lane == 0) {

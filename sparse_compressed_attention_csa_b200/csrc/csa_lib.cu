@@ -129,6 +129,35 @@ csa_status_t launched(const char* what) {
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Launch with programmatic dependent launch allowed (the kernel may start
+// while its predecessor in the stream finishes; it waits for it in
+// griddep_wait() before touching global memory) and, when cluster_x > 1,
+// as clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 int num_sms() {
   static int cached[64];
   int dev = 0;
@@ -182,7 +211,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 2D bf16 tensor map over [rows][inner] row-major, box [box_rows][box_inner],
 // 128-byte swizzle (box_inner * 2 must be 128).
 csa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
-                            uint32_t box_inner, uint32_t box_rows) {
+                            uint32_t box_inner, uint32_t box_rows,
+                            CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {inner, rows};
@@ -190,7 +220,7 @@ csa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, ui
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return CSA_OK;
@@ -253,8 +283,42 @@ bool attn_tc_ok(const csa_params_t* p, csa_dtype_t dtype, bool hca, int n_max) {
 // compiled but not selected.
 int attn_nq(int B, int Tq) { (void)B; (void)Tq; return 2; }
 
+// Clusters of `cluster` attention CTAs that fit on the device at once (0 if
+// the query fails, e.g. without a device).  Cached per (device, size).
+int attn_max_clusters(int cluster) {
+  static std::mutex mu;
+  static int cache[64][kAtMaxSplits + 1];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  int& c = cache[dev][cluster];
+  if (c != 0) return c;
+  const size_t smem = AtLayout<2>::kBytes + 1024;
+  if (set_smem_attr(k_attn_tc<false, 2>, smem, "k_attn_tc") != CSA_OK) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+  cfg.blockDim = dim3(kAtThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = (unsigned)cluster;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_attn_tc<false, 2>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  c = n > 0 ? n : -1;
+  return n;
+}
+
 // KV splits per query token: enough CTAs to cover the SMs, at least one
-// 64-row tile per split.
+// 64-row tile per split, at most one cluster's worth, and no more than lets
+// every cluster of the grid be resident at once (the splits of a token
+// meet at a cluster barrier).
 int attn_splits(const csa_params_t* p, bool hca, int B, int Tq, int n_max) {
   const long long units = (long long)B * Tq * attn_nq(B, Tq);
   const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
@@ -262,6 +326,11 @@ int attn_splits(const csa_params_t* p, bool hca, int B, int Tq, int n_max) {
   const long long max_s = (rows + kAtTile - 1) / kAtTile;
   if (s > max_s) s = max_s;
   if (s > kAtMaxSplits) s = kAtMaxSplits;
+  while (s > 1) {
+    const int fit = attn_max_clusters((int)s);
+    if (fit <= 0 || units <= fit) break;  // unknown (no device): keep s
+    --s;
+  }
   return s < 1 ? 1 : (int)s;
 }
 
@@ -272,8 +341,7 @@ size_t attn_ws_bytes(const csa_params_t* p, csa_dtype_t dtype, bool hca, int B, 
   if (sp == 1) return 0;
   const size_t units = (size_t)B * Tq * sp * attn_nq(B, Tq);
   return round_up(units * kAtHeads * (kAtDim / attn_nq(B, Tq)) * sizeof(float), 256) +
-         round_up(units * 2 * kAtHeads * sizeof(float), 256) +
-         round_up((size_t)B * Tq * attn_nq(B, Tq) * sizeof(int), 256);
+         round_up(units * 2 * kAtHeads * sizeof(float), 256);
 }
 
 }  // namespace
@@ -369,8 +437,10 @@ static csa_status_t launch_index_tc(const void* q_idx, const float* w, const voi
   int chunks = 1;
   if (qblocks * B < num_sms()) chunks = num_sms() / (qblocks * B);
   dim3 grid((unsigned)(qblocks * chunks), (unsigned)B);
-  k_index_scores_tc<QPB, STAGES><<<grid, kIdxTcThreads, smem, s>>>(
-      tk, tq, w, q_pos, n_cmp, Tq, n_max, width, stride, chunks, scores);
+  const cudaError_t e = launch_ex(k_index_scores_tc<QPB, STAGES>, grid, dim3(kIdxTcThreads), smem,
+                                  s, 1, tk, tq, w, q_pos, n_cmp, Tq, n_max, width, stride, chunks,
+                                  scores);
+  if (e != cudaSuccess) return cuda_fail(e, "k_index_scores_tc");
   return launched("k_index_scores_tc");
 }
 
@@ -420,15 +490,15 @@ static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const 
   const int k = p->topk;
   const TopkPlan plan = topk_plan(p, B, Tq, n_max);
   const int chunks = plan.chunks;
+  int* none = nullptr;
   if (chunks == 1) {
-    if (plan.chunk_len == kTopkSmall)
-      k_topk_chunk<256, 8><<<dim3(1, rows), 256, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k,
-                                                          p->width, p->stride, 1, idx_out,
-                                                          nullptr, nullptr);
-    else
-      k_topk_chunk<1024, 16><<<dim3(1, rows), 1024, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k,
-                                                            p->width, p->stride, 1, idx_out,
-                                                            nullptr, nullptr);
+    const cudaError_t e =
+        plan.chunk_len == kTopkSmall
+            ? launch_ex(k_topk_chunk<256, 8>, dim3(1, rows), dim3(256), 0, s, 1, scores, q_pos,
+                        n_cmp, Tq, n_max, k, p->width, p->stride, 1, idx_out, none, none)
+            : launch_ex(k_topk_chunk<1024, 16>, dim3(1, rows), dim3(1024), 0, s, 1, scores, q_pos,
+                        n_cmp, Tq, n_max, k, p->width, p->stride, 1, idx_out, none, none);
+    if (e != cudaSuccess) return cuda_fail(e, "k_topk_chunk");
     return launched("k_topk_chunk");
   }
   if (chunks > 1) {
@@ -439,16 +509,21 @@ static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const 
     CSA_CHECK(check_ptr(ws, "ws"));
     int* cand = (int*)ws;
     int* cand_n = (int*)((char*)ws + round_up((size_t)rows * chunks * (size_t)k * sizeof(int), 256));
-    k_topk_chunk<1024, 16><<<dim3((unsigned)chunks, rows), 1024, 0, s>>>(
-        scores, q_pos, n_cmp, Tq, n_max, k, p->width, p->stride, chunks, idx_out, cand, cand_n);
+    cudaError_t e = launch_ex(k_topk_chunk<1024, 16>, dim3((unsigned)chunks, rows), dim3(1024), 0,
+                              s, 1, scores, q_pos, n_cmp, Tq, n_max, k, p->width, p->stride,
+                              chunks, idx_out, cand, cand_n);
+    if (e != cudaSuccess) return cuda_fail(e, "k_topk_chunk");
     CSA_CHECK(launched("k_topk_chunk"));
     if (plan.merge_cap == kTopkMid)
-      k_topk_merge<256, 16><<<rows, 256, 0, s>>>(scores, n_max, k, chunks, cand, cand_n, idx_out);
+      e = launch_ex(k_topk_merge<256, 16>, dim3(rows), dim3(256), 0, s, 1, scores, n_max, k,
+                    chunks, cand, cand_n, idx_out);
     else if (plan.merge_cap == 2 * kTopkMid)
-      k_topk_merge<512, 16><<<rows, 512, 0, s>>>(scores, n_max, k, chunks, cand, cand_n, idx_out);
+      e = launch_ex(k_topk_merge<512, 16>, dim3(rows), dim3(512), 0, s, 1, scores, n_max, k,
+                    chunks, cand, cand_n, idx_out);
     else
-      k_topk_merge<1024, 16><<<rows, 1024, 0, s>>>(scores, n_max, k, chunks, cand, cand_n,
-                                                   idx_out);
+      e = launch_ex(k_topk_merge<1024, 16>, dim3(rows), dim3(1024), 0, s, 1, scores, n_max, k,
+                    chunks, cand, cand_n, idx_out);
+    if (e != cudaSuccess) return cuda_fail(e, "k_topk_merge");
     return launched("k_topk_merge");
   }
   k_topk_rows<1024><<<rows, 1024, 0, s>>>(scores, q_pos, n_cmp, Tq, n_max, k, p->width,
@@ -567,20 +642,17 @@ static csa_status_t launch_attn_tc_nq(const AttnArgs& g, AttnTcArgs& a, int sp, 
                                       cudaStream_t s) {
   using Lay = AtLayout<NQ>;
   if (sp > 1) {
-    // workspace: partial O | partial (m, l) | arrival counters (zeroed here)
+    // workspace: partial O | partial (m, l)
     const size_t units = (size_t)g.B * g.Tq * sp * NQ;
     const size_t o_bytes = round_up(units * kAtHeads * (kAtDim / NQ) * sizeof(float), 256);
-    const size_t ml_bytes = round_up(units * 2 * kAtHeads * sizeof(float), 256);
     a.part_o = (float*)ws;
     a.part_ml = (float*)((char*)ws + o_bytes);
-    a.arrive = (int*)((char*)ws + o_bytes + ml_bytes);
-    if (cudaMemsetAsync(a.arrive, 0, (size_t)g.B * g.Tq * NQ * sizeof(int), s) != cudaSuccess)
-      return fail(CSA_ERR_CUDA, "cudaMemsetAsync of the split counters failed");
   }
   const size_t smem = Lay::kBytes + 1024;
   CSA_CHECK(set_smem_attr(k_attn_tc<kHca, NQ>, smem, "k_attn_tc"));
   dim3 grid((unsigned)(NQ * sp), (unsigned)(g.B * g.Tq));
-  k_attn_tc<kHca, NQ><<<grid, kAtThreads, smem, s>>>(a, tq, to);
+  const cudaError_t e = launch_ex(k_attn_tc<kHca, NQ>, grid, dim3(kAtThreads), smem, s, sp, a, tq, to);
+  if (e != cudaSuccess) return cuda_fail(e, "k_attn_tc");
   return launched("k_attn_tc");
 }
 
@@ -615,12 +687,12 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   a.out = (__nv_bfloat16*)g.out;
   a.part_o = nullptr;
   a.part_ml = nullptr;
-  a.arrive = nullptr;
   for (int i = 0; i < kAtMaxRope / 2; ++i)
     a.freq[i] = i < g.rope_dim / 2 ? std::pow(g.theta, -2.0 * i / (double)g.rope_dim) : 0.0;
   CUtensorMap tq, to;
   CSA_CHECK(make_tmap_bf16(&tq, g.q, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
-  CSA_CHECK(make_tmap_bf16(&to, g.out, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
+  CSA_CHECK(make_tmap_bf16(&to, g.out, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 32, kAtHeads,
+                           CU_TENSOR_MAP_SWIZZLE_64B));
   if (attn_nq(g.B, g.Tq) == 4) return launch_attn_tc_nq<kHca, 4>(g, a, sp, ws, tq, to, s);
   return launch_attn_tc_nq<kHca, 2>(g, a, sp, ws, tq, to, s);
 }

@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   S& sm = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                 ~static_cast<uintptr_t>(1023));
+  griddep_wait();  // inputs written by the predecessor are visible
+  griddep_launch_dependents();
   const int b = blockIdx.y;
   const int qb = blockIdx.x / chunks, chunk = blockIdx.x % chunks;
   const int t0 = qb * QPB;

@@ -17,6 +17,7 @@
 // fewer than k entries of the row, hence of its chunk.
 #pragma once
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -55,17 +56,17 @@ __device__ __forceinline__ int place_selected(const bool (&sel)[PT], int k, Inde
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
-  unsigned m[PT];
 #pragma unroll
   for (int e = 0; e < PT; ++e) {
-    m[e] = __ballot_sync(0xffffffffu, sel[e]);
-    if (lane == 0) sh.cnt[e * NW + wid] = __popc(m[e]);
+    const unsigned m = __ballot_sync(0xffffffffu, sel[e]);
+    if (lane == 0) sh.cnt[e * NW + wid] = __popc(m);
   }
   const int total = scan_groups(sh);
 #pragma unroll
   for (int e = 0; e < PT; ++e) {
+    const unsigned m = __ballot_sync(0xffffffffu, sel[e]);  // recomputed: fewer live registers
     if (sel[e]) {
-      const int pos = sh.cnt[e * NW + wid] + __popc(m[e] & lt);
+      const int pos = sh.cnt[e * NW + wid] + __popc(m & lt);
       if (pos < k) out[pos] = index_of(e);
     }
   }
@@ -162,26 +163,35 @@ __device__ int block_topk(const uint32_t (&key)[PT], const bool (&valid)[PT], in
       if (remaining == sh.bin_count) break;  // the boundary bin is kept whole
     }
   }
-  // kept: keys above the boundary bin, and the first `remaining` keys (in
-  // index order) of the boundary bin
-  bool gt[PT], eq[PT];
-  unsigned meq[PT];
+  // Kept: keys above the boundary bin, and the first `remaining` keys (in
+  // index order) of the boundary bin.  One scan over the groups, of the
+  // greater and equal counts packed in one int (each total < 2^16), places
+  // them all: a kept candidate's position is the number of kept ones before
+  // it in index order.
+  const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
   for (int e = 0; e < PT; ++e) {
     const uint32_t km = key[e] & mask;
-    gt[e] = valid[e] && km > prefix;
-    eq[e] = valid[e] && km == prefix;
-    meq[e] = __ballot_sync(0xffffffffu, eq[e]);
-    if (lane == 0) sh.cnt[e * NW + wid] = __popc(meq[e]);
+    const unsigned mg = __ballot_sync(0xffffffffu, valid[e] && km > prefix);
+    const unsigned mq = __ballot_sync(0xffffffffu, valid[e] && km == prefix);
+    if (lane == 0) sh.cnt[e * NW + wid] = (__popc(mg) << 16) | __popc(mq);
   }
   scan_groups(sh);
-  const unsigned lt = (1u << lane) - 1u;
-  bool sel[PT];
 #pragma unroll
-  for (int e = 0; e < PT; ++e)
-    sel[e] = gt[e] || (eq[e] && sh.cnt[e * NW + wid] + __popc(meq[e] & lt) < remaining);
-  __syncthreads();  // every thread has read the tie ranks before cnt is reused
-  place_selected<NT, PT>(sel, k, index_of, out, sh);
+  for (int e = 0; e < PT; ++e) {
+    const uint32_t km = key[e] & mask;
+    const bool g = valid[e] && km > prefix, q = valid[e] && km == prefix;
+    const unsigned mg = __ballot_sync(0xffffffffu, g);
+    const unsigned mq = __ballot_sync(0xffffffffu, q);
+    const int before = sh.cnt[e * NW + wid];
+    const int g_before = before >> 16, q_before = before & 0xffff;
+    const int q_rank = q_before + __popc(mq & lt);  // rank among the boundary keys
+    if (g || (q && q_rank < remaining)) {
+      // kept before this one: greater ones, plus boundary ones of rank < remaining
+      const int pos = g_before + __popc(mg & lt) + min(q_rank, remaining);
+      if (pos < k) out[pos] = index_of(e);
+    }
+  }
   return k;
 }
 
@@ -196,18 +206,27 @@ __global__ void __launch_bounds__(NT)
                  int n_chunks, int* __restrict__ idx_out, int* __restrict__ cand,
                  int* __restrict__ cand_n) {
   __shared__ TopkShared<NT, PT> sh;
+  sm100::griddep_wait();  // the scores of the predecessor are visible
+  sm100::griddep_launch_dependents();
   const int c = blockIdx.x, row = blockIdx.y;
   const int b = row / Tq;
-  const int nv = min(n_visible(q_pos[row], n_cmp[b], width, stride), n_max);
   const int base = c * NT * PT + (int)threadIdx.x;
   const float* s = scores + (size_t)row * n_max;
+  // the row's scores are loaded up to n_max (in bounds) without waiting for
+  // the visible count, then masked
+  float v[PT];
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    const int j = base + e * NT;
+    v[e] = j < n_max ? s[j] : 0.f;
+  }
+  const int nv = min(n_visible(q_pos[row], n_cmp[b], width, stride), n_max);
   uint32_t key[PT];
   bool valid[PT];
 #pragma unroll
   for (int e = 0; e < PT; ++e) {
-    const int j = base + e * NT;
-    valid[e] = j < nv;
-    key[e] = valid[e] ? float_key(s[j]) : 0u;
+    valid[e] = base + e * NT < nv;
+    key[e] = valid[e] ? float_key(v[e]) : 0u;
   }
   int* out = n_chunks == 1 ? idx_out + (size_t)row * k : cand + ((size_t)row * n_chunks + c) * k;
   const int cnt = block_topk<NT, PT>(key, valid, k, [&](int e) { return base + e * NT; }, out, sh);
@@ -226,6 +245,8 @@ __global__ void __launch_bounds__(NT)
                  int* __restrict__ idx_out) {
   __shared__ TopkShared<NT, PT> sh;
   __shared__ int offs[65];
+  sm100::griddep_wait();
+  sm100::griddep_launch_dependents();
   const int row = blockIdx.x;
   if (threadIdx.x == 0) {
     int acc = 0;
