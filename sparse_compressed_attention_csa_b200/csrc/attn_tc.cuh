@@ -484,23 +484,34 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int g0 = r_lo + i * kAtTile;  // list index of row 0 of the tile
-      float z[64];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r[32];
-        tmem_ld32(t_s + lane_base + (uint32_t)(sb * 64 + hh * 32), r);
+      float z[64];  // raw logits q.k (scaled to the log2 domain below)
+      {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(t_s + lane_base + (uint32_t)(sb * 64), ra);
+        tmem_ld32(t_s + lane_base + (uint32_t)(sb * 64 + 32), rb);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) z[hh * 32 + e] = __uint_as_float(r[e]) * a.scale_log2;
+        for (int e = 0; e < 32; ++e) {
+          z[e] = __uint_as_float(ra[e]);
+          z[32 + e] = __uint_as_float(rb[e]);
+        }
       }
-      float mt = -INFINITY;
+      // rows of the tile outside the split, padding between the selected and
+      // the window rows, and padding at the end are masked; most tiles have
+      // none
+      const int g1 = g0 + kAtTile - 1;
+      if (!(g1 < r_hi && (g1 < n_sel || (g0 >= ps && g1 < pe)))) {
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const int g = g0 + e;
-        const bool valid = g < r_hi && (g < n_sel || (g >= ps && g < pe));
-        if (!valid) z[e] = -INFINITY;
-        mt = fmaxf(mt, z[e]);
+        for (int e = 0; e < 64; ++e) {
+          const int g = g0 + e;
+          const bool valid = g < r_hi && (g < n_sel || (g >= ps && g < pe));
+          if (!valid) z[e] = -INFINITY;
+        }
       }
+      float zmax = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) zmax = fmaxf(zmax, z[e]);
+      const float mt = zmax * a.scale_log2;  // the scale is positive: max commutes
       if (mt > m_run + kAtRescaleLog2 || m_run == -INFINITY) {
         if (i > 0) {
           // O holds P V of earlier tiles: wait for the last PV, then rescale
@@ -529,9 +540,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
       uint32_t pk[32];
       float psum = 0.f;
+      const float neg_m = -m_run;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = ex2_approx(z[2 * e] - m_run), p1 = ex2_approx(z[2 * e + 1] - m_run);
+        const float p0 = ex2_approx(fmaf(z[2 * e], a.scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(z[2 * e + 1], a.scale_log2, neg_m));
         __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
         const float2 back = __bfloat1622float2(pb);
         psum += back.x + back.y;
@@ -632,9 +645,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       for (int ck = 0; ck < 4; ++ck, ++n) {
         const int chunk = chunk_of[ck];
         const int slot = n % kSlots;
-        okp = mbar_wait_backoff(&sm.empty[slot], ((uint32_t)(n / kSlots) & 1u) ^ 1u, abortp);
+        okp = mbar_wait(&sm.empty[slot], ((uint32_t)(n / kSlots) & 1u) ^ 1u, abortp);
         if (okp && !staged && slot >= kSlots - Lay::kQStage) {  // slot still holds q staging
-          okp = mbar_wait_backoff(&sm.q_ready, 0, abortp);
+          okp = mbar_wait(&sm.q_ready, 0, abortp);
           staged = true;
         }
         if (!okp) break;
@@ -683,20 +696,47 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     int pv_next = 0;  // next tile whose PV is still to be issued
     for (int i = 0; i < ntile && okm; ++i) {
       const int sb = i & 1;
-      if (i >= 2) {  // P(i-2) lives in S[sb]: its PV must have finished
-        if (pv_next <= i - 2) okm = issue_pv(pv_next++);
+      if (i >= 2 && pv_next <= i - 2) {
+        // P(i-2) lives in S[sb]: its PV is issued before S(i) overwrites it.
+        // MMAs of one thread execute in issue order, so the PV reads P before
+        // the QK MMAs below write that TMEM; no wait for its completion.
+        okm = issue_pv(pv_next++);
         if (!okm) break;
-        okm = mbar_wait(&sm.pv_done[sb], (uint32_t)((i - 2) >> 1) & 1u, abortp);
-        if (!okm) break;
-        tc_fence_after();
       }
       // S(i) = Q K_i^T over the four 128-dim chunks (others first)
       for (int ck = 0; ck < 4 && okm; ++ck, ++n) {
         const int chunk = chunk_of[ck];
         const bool own = ck >= 4 - kOwn;
         const int slot = n % kSlots;
-        okm = mbar_wait(&sm.full[slot], (uint32_t)(n / kSlots) & 1u, abortp);
         if (own) own_slot[sb][ck - (4 - kOwn)] = slot;
+        // wait for the chunk; meanwhile the previous tile's PV goes in as
+        // soon as its P is ready (so that its V slots are released early)
+        {
+          const uint32_t fph = (uint32_t)(n / kSlots) & 1u;
+          if (!mbar_try_wait(&sm.full[slot], fph)) {
+            const uint64_t t_start = globaltimer();
+            for (uint32_t it = 1;; ++it) {
+              if (pv_next == i - 1 &&
+                  mbar_try_wait(&sm.p_full[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u)) {
+                okm = issue_pv(pv_next++);
+                if (!okm) break;
+              }
+              if (mbar_try_wait(&sm.full[slot], fph)) break;
+              if ((it & 63u) == 0u) {
+                if (*abortp) {
+                  okm = false;
+                  break;
+                }
+                if (globaltimer() - t_start > kWaitLimitNs) {
+                  *abortp = 1;
+                  report_error(CSA_ERR_DEVICE_TIMEOUT);
+                  okm = false;
+                  break;
+                }
+              }
+            }
+          }
+        }
         if (!okm) break;
         // written by cp.async (generic proxy), read by the MMA (async proxy)
         fence_proxy_async();

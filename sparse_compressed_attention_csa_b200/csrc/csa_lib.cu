@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -189,6 +190,11 @@ csa_status_t set_smem_attr(K* kernel, size_t bytes, const char* name) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes);
   if (e != cudaSuccess) return cuda_fail(e, name);
+  // these kernels live on shared memory: ask for the largest carveout, so
+  // that occupancy queries and launches both see every CTA that fits
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return cuda_fail(e, name);
   if (n_done < 256) done[n_done++] = Entry{(const void*)kernel, dev};
   return CSA_OK;
 }
@@ -230,8 +236,10 @@ size_t scores_bytes(int B, int Tq, int n_max) {
   return round_up((size_t)B * Tq * (size_t)n_max * sizeof(float), 256);
 }
 
-// Top-k plan.  A block holds its candidates in registers: 2048 (256 x 8) or
-// 16384 (1024 x 16) entries.  One block per row when the row fits; two
+// Top-k plan.  A block holds its candidates in registers: 2048 (256 x 8),
+// 4096 (256 x 16) or 16384 (1024 x 16) entries.  Few rows of up to 32768
+// entries: one cluster of 4096-entry CTAs per row.  Else one block per row
+// when the row fits; two
 // stages (per-chunk top-k into a candidate list, then one merge block per
 // row over the concatenated candidates) for longer rows when the merge fits
 // one block (4096, 8192 or 16384 candidates); else the generic
@@ -242,22 +250,27 @@ struct TopkPlan {
   int chunks;     // 0: generic; 1: single stage; >1: chunk + merge
   int chunk_len;  // entries per chunk block
   int merge_cap;  // candidates per merge block
+  int cluster;    // > 1: one cluster of this many 4096-entry CTAs per row
 };
 constexpr int kTopkSmall = 256 * 8, kTopkMid = 256 * 16, kTopkBig = 1024 * 16;
 
 TopkPlan topk_plan(const csa_params_t* p, int B, int Tq, int n_max) {
-  (void)B;
-  (void)Tq;
+  const long long rows = (long long)B * Tq;
   const long long k = p->topk;
-  if (n_max <= kTopkSmall) return {1, kTopkSmall, 0};
-  if (n_max <= kTopkBig) return {1, kTopkBig, 0};
+  // few long rows: a cluster of CTAs per row, so that the SMs share the rows
+  if (n_max > kTopkMid && n_max <= kTopkMaxCluster * kTopkMid && 2 * rows <= num_sms()) {
+    const int c = (n_max + kTopkMid - 1) / kTopkMid;
+    if (rows * c <= num_sms()) return {1, kTopkMid, 0, c};
+  }
+  if (n_max <= kTopkSmall) return {1, kTopkSmall, 0, 0};
+  if (n_max <= kTopkBig) return {1, kTopkBig, 0, 0};
   const long long c = (n_max + kTopkBig - 1) / kTopkBig;
   if (c <= 64 && c * k <= kTopkBig) {
     const long long cand = c * k;
     return {(int)c, kTopkBig,
-            cand <= kTopkMid ? kTopkMid : (cand <= 2 * kTopkMid ? 2 * kTopkMid : kTopkBig)};
+            cand <= kTopkMid ? kTopkMid : (cand <= 2 * kTopkMid ? 2 * kTopkMid : kTopkBig), 0};
   }
-  return {0, 0, 0};
+  return {0, 0, 0, 0};
 }
 
 size_t topk_ws_bytes(const csa_params_t* p, int B, int Tq, int n_max) {
@@ -434,8 +447,13 @@ static csa_status_t launch_index_tc(const void* q_idx, const float* w, const voi
   const size_t smem = sizeof(IdxTcSmem<QPB, STAGES>) + 1024;
   CSA_CHECK(set_smem_attr(k_index_scores_tc<QPB, STAGES>, smem, "k_index_scores_tc"));
   const int qblocks = (Tq + QPB - 1) / QPB;
+  // key ranges per query block: enough CTAs to fill every SM with as many
+  // CTAs as its 228 KB of shared memory holds (1 KB reserved per CTA); the
+  // registers (192 threads x at most 168) allow two
+  const int per_sm = 2 * (smem + 1024) <= 228 * 1024 ? 2 : 1;
+  const int slots = per_sm * num_sms();
   int chunks = 1;
-  if (qblocks * B < num_sms()) chunks = num_sms() / (qblocks * B);
+  if (qblocks * B < slots) chunks = slots / (qblocks * B);
   dim3 grid((unsigned)(qblocks * chunks), (unsigned)B);
   const cudaError_t e = launch_ex(k_index_scores_tc<QPB, STAGES>, grid, dim3(kIdxTcThreads), smem,
                                   s, 1, tk, tq, w, q_pos, n_cmp, Tq, n_max, width, stride, chunks,
@@ -454,7 +472,7 @@ static csa_status_t index_scores_impl(const csa_params_t* p, csa_dtype_t dtype, 
   if (dtype == CSA_BF16 && H_I == kIdxTcHeads && d_I == kIdxTcDim &&
       (long long)B * n_max >= kIdxTcKeys) {
     if (Tq == 1)
-      return launch_index_tc<1, 6>(q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, p->width,
+      return launch_index_tc<1, 2>(q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, p->width,
                                    p->stride, scores, s);
     if ((long long)B * Tq >= 2)
       return launch_index_tc<2, 2>(q_idx, w, k_idx, q_pos, n_cmp, B, Tq, n_max, p->width,
@@ -491,6 +509,13 @@ static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const 
   const TopkPlan plan = topk_plan(p, B, Tq, n_max);
   const int chunks = plan.chunks;
   int* none = nullptr;
+  if (plan.cluster > 1) {
+    const cudaError_t e =
+        launch_ex(k_topk_cluster<256, 16>, dim3((unsigned)plan.cluster, rows), dim3(256), 0, s,
+                  plan.cluster, scores, q_pos, n_cmp, Tq, n_max, k, p->width, p->stride, idx_out);
+    if (e != cudaSuccess) return cuda_fail(e, "k_topk_cluster");
+    return launched("k_topk_cluster");
+  }
   if (chunks == 1) {
     const cudaError_t e =
         plan.chunk_len == kTopkSmall

@@ -13,6 +13,9 @@
 // accumulators, warps 2-5 read the accumulators back (one TMEM lane = one
 // key per thread) and write the scores.  Every product and sum is exact for
 // integer-valued inputs with power-of-two weights (partial sums < 2^24).
+// Decode runs two CTAs per SM with 2-stage rings (measured faster than one
+// CTA with a 6-stage ring: the two interleave each other's epilogue and MMA
+// latency).
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -206,5 +209,6 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
     tmem_dealloc(tmem, kCols);
   }
 }
+
 
 }  // namespace csa

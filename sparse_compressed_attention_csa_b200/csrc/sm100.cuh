@@ -77,28 +77,6 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
   }
 }
 
-// As mbar_wait, but sleeps between polls: for threads that run far ahead of
-// their consumer (copy producers), so that their polling does not take issue
-// slots from the warps on the critical path.
-__device__ __noinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity,
-                                               volatile int* abort_flag,
-                                               uint64_t limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(128);
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0u) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > limit_ns) {
-        *abort_flag = 1;
-        report_error(CSA_ERR_DEVICE_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -282,4 +282,220 @@ __global__ void __launch_bounds__(NT)
   for (int i = cnt + threadIdx.x; i < k; i += NT) out[i] = -1;
 }
 
+// ---------------------------------------------------------------------------
+// Few long rows: one thread-block cluster of C CTAs per row (C = gridDim.x,
+// at most kTopkMaxCluster), CTA c holding entries [c * NT * PT, (c + 1) * NT
+// * PT) striped as above.  The CTAs exchange, through distributed shared
+// memory, their valid counts and AND/OR of keys, each radix pass's 256-bin
+// histogram and, at the end, their counts of greater and boundary keys; one
+// cluster barrier per exchange.  Every CTA then takes the same decisions on
+// the same totals and places its kept entries after those of the lower
+// ranks, so the row's output is the single-block result.
+constexpr int kTopkMaxCluster = 8;
+
+template <int NT, int PT>
+struct TopkClusterShared {
+  TopkShared<NT, PT> loc;
+  unsigned xh[2][kTopkMaxCluster][256];  // per-pass histograms of every rank (double buffer)
+  int xv[3][kTopkMaxCluster][3];         // small per-rank values of the three exchanges
+};
+
+// Stores v at the same shared-memory offset as `local` in cluster CTA `rank`.
+__device__ __forceinline__ void dsmem_store(const void* local, uint32_t rank, uint32_t v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(ra)
+               : "r"(sm100::smem_u32(local)), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
+}
+
+template <int NT, int PT>
+__global__ void __launch_bounds__(NT)
+    k_topk_cluster(const float* __restrict__ scores, const int* __restrict__ q_pos,
+                   const int* __restrict__ n_cmp, int Tq, int n_max, int k, int width,
+                   int stride, int* __restrict__ idx_out) {
+  static_assert(NT >= 256, "bin scan needs 256 threads");
+  constexpr int NW = NT / 32;
+  __shared__ TopkClusterShared<NT, PT> sh;
+  sm100::griddep_wait();  // the scores of the predecessor are visible
+  sm100::griddep_launch_dependents();
+  const int C = (int)gridDim.x;
+  const int c = (int)blockIdx.x;  // cluster rank: the cluster spans the grid's x
+  const int row = blockIdx.y;
+  const int b = row / Tq;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int base = c * NT * PT + (int)threadIdx.x;
+  const float* s = scores + (size_t)row * n_max;
+  int* out = idx_out + (size_t)row * k;
+  float v[PT];
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    const int j = base + e * NT;
+    v[e] = j < n_max ? s[j] : 0.f;
+  }
+  const int nv = min(n_visible(q_pos[row], n_cmp[b], width, stride), n_max);
+  uint32_t key[PT];
+  bool valid[PT];
+  int nv_local = 0;
+  uint32_t k_and = 0xffffffffu, k_or = 0u;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    valid[e] = base + e * NT < nv;
+    key[e] = valid[e] ? float_key(v[e]) : 0u;
+    if (valid[e]) {
+      ++nv_local;
+      k_and &= key[e];
+      k_or |= key[e];
+    }
+  }
+  // ---- exchange 0: valid counts and AND / OR of the keys
+  int n_mine;
+  block_inclusive_scan(nv_local, sh.loc.scan, &n_mine);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    k_and &= __shfl_xor_sync(0xffffffffu, k_and, o);
+    k_or |= __shfl_xor_sync(0xffffffffu, k_or, o);
+  }
+  if (lane == 0) {
+    sh.loc.red_and[wid] = k_and;
+    sh.loc.red_or[wid] = k_or;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < C) {
+    uint32_t a = 0xffffffffu, o = 0u;
+    for (int w = 0; w < NW; ++w) {
+      a &= sh.loc.red_and[w];
+      o |= sh.loc.red_or[w];
+    }
+    const uint32_t r = threadIdx.x;
+    dsmem_store(&sh.xv[0][c][0], r, (uint32_t)n_mine);
+    dsmem_store(&sh.xv[0][c][1], r, a);
+    dsmem_store(&sh.xv[0][c][2], r, o);
+  }
+  sm100::cluster_sync_all();
+  int n_valid = 0, valid_before = 0;
+  k_and = 0xffffffffu;
+  k_or = 0u;
+  for (int r = 0; r < C; ++r) {
+    const int n = sh.xv[0][r][0];
+    n_valid += n;
+    valid_before += r < c ? n : 0;
+    if (n > 0) {
+      k_and &= (uint32_t)sh.xv[0][r][1];
+      k_or |= (uint32_t)sh.xv[0][r][2];
+    }
+  }
+  if (c == 0)
+    for (int i = min(n_valid, k) + (int)threadIdx.x; i < k; i += NT) out[i] = -1;
+  if (n_valid <= k) {  // keep every valid entry
+    place_selected<NT, PT>(valid, k - valid_before, [&](int e) { return base + e * NT; },
+                           out + valid_before, sh.loc);
+    return;  // no exchange follows: no CTA writes into another's memory any more
+  }
+  // ---- radix select on the row's totals
+  const uint32_t diff = k_and ^ k_or;
+  uint32_t prefix, mask;
+  int remaining = k;
+  if (diff == 0u) {
+    prefix = k_and;
+    mask = 0xffffffffu;
+  } else {
+    int hi = 31 - __clz(diff);
+    mask = hi == 31 ? 0u : (0xffffffffu << (hi + 1));
+    prefix = k_and & mask;
+    int pass = 0;
+#pragma unroll 1
+    while (hi >= 0) {
+      const int lo = max(hi - 7, 0);
+      const uint32_t dmask = ((hi - lo == 31) ? 0xffffffffu : ((1u << (hi - lo + 1)) - 1u));
+      for (int i = threadIdx.x; i < 256; i += NT) sh.loc.hist[i] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < PT; ++e)
+        if (valid[e] && (key[e] & mask) == prefix)
+          atomicAdd(&sh.loc.hist[(key[e] >> lo) & dmask], 1u);
+      __syncthreads();
+      unsigned (*xh)[256] = sh.xh[pass & 1];
+      if (threadIdx.x < 256) {
+        const unsigned h = sh.loc.hist[threadIdx.x];
+        for (int r = 0; r < C; ++r) dsmem_store(&xh[c][threadIdx.x], (uint32_t)r, h);
+      }
+      sm100::cluster_sync_all();
+      if (threadIdx.x < 256) {
+        const int bin = 255 - (int)threadIdx.x;
+        int h = 0;
+        for (int r = 0; r < C; ++r) h += (int)xh[r][bin];
+        int x = h;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += n;
+        }
+        if (lane == 31) sh.loc.scan[wid] = x;
+        asm volatile("bar.sync 3, 256;" ::: "memory");
+        int off = 0;
+        for (int w = 0; w < wid; ++w) off += sh.loc.scan[w];
+        const int incl = off + x, excl = incl - h;
+        if (incl >= remaining && excl < remaining) {
+          sh.loc.prefix = prefix | ((uint32_t)bin << lo);
+          sh.loc.remaining = remaining - excl;
+          sh.loc.bin_count = h;
+        }
+      }
+      __syncthreads();
+      prefix = sh.loc.prefix;
+      remaining = sh.loc.remaining;
+      mask |= dmask << lo;
+      hi = lo - 1;
+      ++pass;
+      if (remaining == sh.loc.bin_count) break;  // the boundary bin is kept whole
+    }
+  }
+  // ---- exchange 2: greater and boundary counts of every rank
+  int g_mine = 0, q_mine = 0;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    const uint32_t km = key[e] & mask;
+    g_mine += (valid[e] && km > prefix) ? 1 : 0;
+    q_mine += (valid[e] && km == prefix) ? 1 : 0;
+  }
+  int g_tot, q_tot;
+  block_inclusive_scan(g_mine, sh.loc.scan, &g_tot);
+  block_inclusive_scan(q_mine, sh.loc.scan, &q_tot);
+  if ((int)threadIdx.x < C) {
+    dsmem_store(&sh.xv[2][c][0], threadIdx.x, (uint32_t)g_tot);
+    dsmem_store(&sh.xv[2][c][1], threadIdx.x, (uint32_t)q_tot);
+  }
+  sm100::cluster_sync_all();
+  int g_rank = 0, q_rank0 = 0;  // greater / boundary keys in the lower ranks
+  for (int r = 0; r < c; ++r) {
+    g_rank += sh.xv[2][r][0];
+    q_rank0 += sh.xv[2][r][1];
+  }
+  // ---- placement, as in block_topk, offset by the lower ranks
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    const uint32_t km = key[e] & mask;
+    const unsigned mg = __ballot_sync(0xffffffffu, valid[e] && km > prefix);
+    const unsigned mq = __ballot_sync(0xffffffffu, valid[e] && km == prefix);
+    if (lane == 0) sh.loc.cnt[e * NW + wid] = (__popc(mg) << 16) | __popc(mq);
+  }
+  scan_groups(sh.loc);
+#pragma unroll
+  for (int e = 0; e < PT; ++e) {
+    const uint32_t km = key[e] & mask;
+    const bool g = valid[e] && km > prefix, q = valid[e] && km == prefix;
+    const unsigned mg = __ballot_sync(0xffffffffu, g);
+    const unsigned mq = __ballot_sync(0xffffffffu, q);
+    const int before = sh.loc.cnt[e * NW + wid];
+    const int g_before = g_rank + (before >> 16), q_before = q_rank0 + (before & 0xffff);
+    const int q_rank = q_before + __popc(mq & lt);
+    if (g || (q && q_rank < remaining)) {
+      const int pos = g_before + __popc(mg & lt) + min(q_rank, remaining);
+      if (pos < k) out[pos] = base + e * NT;
+    }
+  }
+}
+
 }  // namespace csa

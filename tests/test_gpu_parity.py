@@ -168,6 +168,26 @@ def test_index_scores_bit_exact():
         assert np.array_equal(got[tq, :nv], want[tq, :nv]), tq
 
 
+def test_index_scores_decode_ragged_visibility():
+    # one query per sequence at different positions: the decode indexer skips
+    # tiles past each sequence's visible entries and switches query blocks
+    # where a CTA's range of tiles crosses a sequence boundary
+    wl = W.CSA_DECODE_64K.replace(B=7, T=20000, seed=32)
+    data = W.generate(wl)
+    data["q_pos"] = np.array([[19999], [5000], [129], [7], [3000], [19998], [0]], dtype=np.int32)
+    p = params_of(wl)
+    t = {k: dev(data[k]) for k in ("q_idx", "w", "k_idx", "q_pos", "n_cmp")}
+    sc = torch.full((wl.B, 1, wl.n_cmp), float("nan"), dtype=torch.float32, device="cuda")
+    csa_index_scores(p, t["q_idx"], t["w"], t["k_idx"], t["q_pos"], t["n_cmp"], sc)
+    torch.cuda.synchronize()
+    got = sc.cpu().numpy().astype(np.float64)
+    for b in range(wl.B):
+        nv = oracle.n_visible(int(data["q_pos"][b, 0]), wl.n_cmp, wl.width, wl.stride)
+        want = oracle.index_scores(f64(data, "q_idx", b), data["w"][b], f64(data, "k_idx", b))
+        assert np.array_equal(got[b, 0, :nv], want[0, :nv]), b
+        assert np.all(np.isnan(got[b, 0, nv:])), b  # nothing written past the visible entries
+
+
 def _adversarial_rows(rng, n):
     return [
         np.zeros(n),                                        # all tied
@@ -180,22 +200,30 @@ def _adversarial_rows(rng, n):
     ]
 
 
-# (entries, k, rows): one block per row up to 16384 entries, else chunks of
-# 16384 and a merge block of 4096, 8192 or 16384 candidates
-@pytest.mark.parametrize("n,k,rows", [
-    (5000, 1024, 7),      # one 16384-entry block per row
-    (1500, 64, 20),       # one 2048-entry block per row
-    (40000, 1024, 7),     # 3 chunks, merge of 3072 candidates
-    (70000, 1024, 7),     # 5 chunks, merge of 5120
-    (70000, 3000, 3),     # 5 chunks, merge of 15000
+# (entries, k, rows, visible): few rows of up to 32768 entries take a cluster
+# of 4096-entry CTAs per row; otherwise one block per row up to 16384
+# entries, else chunks of 16384 and a merge block of 4096, 8192 or 16384
+# candidates
+@pytest.mark.parametrize("n,k,rows,visible", [
+    (5000, 1024, 7, None),     # cluster of 2
+    (9000, 64, 3, None),       # cluster of 3
+    (16383, 1024, 5, None),    # cluster of 4
+    (30000, 1024, 7, None),    # cluster of 8
+    (20000, 1024, 3, 700),     # cluster of 5, fewer visible than k
+    (5000, 1024, 84, None),    # one 16384-entry block per row
+    (1500, 64, 20, None),      # one 2048-entry block per row
+    (40000, 1024, 7, None),    # 3 chunks, merge of 3072 candidates
+    (70000, 1024, 7, None),    # 5 chunks, merge of 5120
+    (70000, 3000, 3, None),    # 5 chunks, merge of 15000
 ])
-def test_topk_select_adversarial_scores(n, k, rows):
+def test_topk_select_adversarial_scores(n, k, rows, visible):
     rng = np.random.default_rng(29 + n + k + rows)
     base = _adversarial_rows(rng, n)
     scores = np.stack([base[r % len(base)] for r in range(rows)]).astype(np.float32)[:, None, :]
     B = scores.shape[0]
     p = Params(topk=k, width=8, stride=4)
-    q_pos = np.full((B, 1), 4 * (n - 1) + 7, dtype=np.int32)   # every entry visible
+    nv = n if visible is None else visible
+    q_pos = np.full((B, 1), 4 * (nv - 1) + 7, dtype=np.int32)   # entries 0 .. nv-1 visible
     n_cmp = np.full((B,), n, dtype=np.int32)
     idx = torch.empty((B, 1, k), dtype=torch.int32, device="cuda")
     nb = csa_workspace_size(p, CSA_OP_TOPK_SELECT, B, 1, n)
@@ -204,7 +232,7 @@ def test_topk_select_adversarial_scores(n, k, rows):
     torch.cuda.synchronize()
     got = idx.cpu().numpy()
     for b in range(B):
-        want = oracle.topk_select(scores[b, 0].astype(np.float64), n, k)
+        want = oracle.topk_select(scores[b, 0].astype(np.float64), nv, k)
         assert np.array_equal(got[b, 0], want), b
 
 
