@@ -42,6 +42,33 @@ UNIT = "query-heads/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+TRAFFIC_DIR = os.path.join(ROOT, "profiles")
+
+
+def _source_digest():
+    """Digest of the kernel sources: recorded DRAM traffic is reported only
+    for the kernels it was captured from."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_compressed_attention_csa_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _recorded_traffic(wl):
+    """DRAM bytes per launch of each kernel group (dram__bytes_read.sum +
+    dram__bytes_write.sum of one ncu capture, profiles/dram_traffic_<workload>
+    .json), or {} when absent or captured from other kernel sources."""
+    try:
+        rec = json.load(open(os.path.join(TRAFFIC_DIR, f"dram_traffic_{wl.name}.json")))
+    except (OSError, ValueError):
+        return {}
+    if rec.get("source_digest") != _source_digest():
+        return {}
+    return dict(rec.get("bytes_per_launch", {}))
 
 
 def _args():
@@ -55,6 +82,8 @@ def _args():
                          "hca_decode_bs16_ctx131072 or csa_prefill_T8192")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the workload's tokens per sequence (profiling cases)")
     ap.add_argument("--flush-mib", type=int, default=256,
                     help="L2 flush size per side (0: no flush; only for profiling, where the "
                          "profiler flushes caches itself)")
@@ -65,14 +94,16 @@ def _args():
     return a
 
 
-def _workload(name, batch=0):
+def _workload(name, batch=0, seq_len=0):
     from sparse_compressed_attention_csa_b200 import workloads as W
     if name not in W.WORKLOADS or W.WORKLOADS[name].dtype != "bf16":
         raise SystemExit(f"unknown workload {name}; choose from "
                          f"{[n for n, w in W.WORKLOADS.items() if w.dtype == 'bf16']}")
     wl = W.WORKLOADS[name]
     if batch and batch != wl.B:
-        wl = wl.replace(B=batch, name=f"{name}_b{batch}")
+        wl = wl.replace(B=batch, name=f"{wl.name}_b{batch}")
+    if seq_len and seq_len != wl.T:
+        wl = wl.replace(T=seq_len, name=f"{wl.name}_T{seq_len}")
     return wl
 
 
@@ -266,7 +297,7 @@ def _oracle_sample(wl):
 def run_reference(args, rank):
     if rank != 0:
         return 0
-    wl = _workload(args.workload, args.batch)
+    wl = _workload(args.workload, args.batch, args.seq_len)
     step, qh, desc = _oracle_sample(wl)
     for _ in range(args.warmup):
         step()
@@ -326,7 +357,7 @@ def run_cuda(args, rank, world, local):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    wl = _workload(args.workload, args.batch)
+    wl = _workload(args.workload, args.batch, args.seq_len)
     data = W.generate(wl)
 
     def todev(a):
@@ -515,6 +546,7 @@ def run_cuda(args, rank, world, local):
         tc = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
         work = algorithmic_work(wl)
         kernel_ms = {name: bd[i] for i, (name, _) in enumerate(groups)}
+        traffic = _recorded_traffic(wl)
         rl = {}
         for k, ms in kernel_ms.items():
             b, f = work[k]["bytes"], work[k]["flops"]
@@ -528,7 +560,7 @@ def run_cuda(args, rank, world, local):
                      "frac": (tfl / tc) if tensor else (gbs / hbm),
                      "algorithmic_bytes": b, "flops": f, "ms": ms,
                      "hbm_frac": gbs / hbm, "tensor_frac": tfl / tc if f else 0.0,
-                     "traffic": None, "peak_source": src + " burst"}
+                     "traffic": traffic.get(k), "peak_source": src + " burst"}
         dom = max(kernel_ms, key=kernel_ms.get)
         line = {
             "metric": _metric(wl), "value": value, "unit": UNIT, "n_gpus": world,
