@@ -339,6 +339,23 @@ def cpu_baseline(wl, budget_s=12.0):
             "sample": f"{n} step(s) of: {desc}; {el:.1f} s"}
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of every rank's x (all ranks call it, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, slowest_ms: float) -> float:
+    """Whole-job throughput of `world` replicas: every rank's units over the
+    slowest rank's time (weak scaling)."""
+    return world * units_per_rank / (slowest_ms * 1e-3)
+
+
 # ------------------------------------------------------------------ CUDA arm
 def run_cuda(args, rank, world, local):
     import numpy as np
@@ -477,12 +494,9 @@ def run_cuda(args, rank, world, local):
     step_ms = tot / args.steps
     n_bd = min(args.steps, 200)
     bd = breakdown(n_bd)
-    t_max = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    step_ms_max = float(t_max.item())
+    step_ms_max = max_over_ranks(step_ms, world, dev)
     qh_per_step = wl.B * wl.Tq * wl.n_heads
-    value = world * qh_per_step / (step_ms_max * 1e-3)
+    value = job_throughput(qh_per_step, world, step_ms_max)
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host
     h2d_keys = {"csa_decode": ("q", "q_idx", "w", "q_pos"), "hca_decode": ("q", "q_pos"),
@@ -530,11 +544,9 @@ def run_cuda(args, rank, world, local):
     if world > 1:
         dist.barrier()
     e2e_ms = sum(e2e_step() for _ in range(n_e2e)) / n_e2e
-    e_max = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    e2e_value = job_throughput(qh_per_step, world, max_over_ranks(e2e_ms, world, dev))
     if world > 1:
-        dist.all_reduce(e_max, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_value = world * qh_per_step / (float(e_max.item()) * 1e-3)
     L.csa_poll_device_error(stream)
 
     if rank == 0:

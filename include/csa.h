@@ -46,7 +46,12 @@
  *   kernel (a bounded wait that ran out) are recorded in a per-device error
  *   word that csa_poll_device_error() reads and clears.
  * Asynchrony: every compute call only enqueues work on `stream`; calls on
- *   different streams are independent.
+ *   different streams are independent.  The tensor-core kernels launch with
+ *   programmatic dependent launch: one may start while its predecessor on
+ *   the stream is finishing, but it waits for that predecessor to complete
+ *   (and its writes to be visible) before its first access to global
+ *   memory, so stream order holds for all data.  The attention calls with
+ *   few query tokens launch thread-block clusters.
  */
 #ifndef CSA_H_
 #define CSA_H_
