@@ -46,13 +46,13 @@ TRAFFIC_DIR = os.path.join(ROOT, "profiles")
 
 
 def _source_digest():
-    """Digest of the kernel sources: recorded DRAM traffic is reported only
-    for the kernels it was captured from."""
+    """Digest of the device code (the kernel headers): recorded DRAM traffic
+    is reported only for the kernels it was captured from."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_compressed_attention_csa_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
+        if f.endswith(".cuh"):
             h.update(f.encode())
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]

@@ -33,6 +33,8 @@
  *   Element type of the "value" arrays (x, gate, q, kv caches, indexer
  *   q/k, out) is the call's csa_dtype_t; weights, sink and scores are fp32;
  *   positions, counts and indices are int32.
+ * Sizes: B >= 1 sequences of Tq >= 1 query tokens with B * Tq <= 65535, and
+ *   n_max >= 0 entries per sequence; otherwise CSA_ERR_UNSUPPORTED_SHAPE.
  * Positions: token t of a sequence sits at position t (the first token at
  *   0).  Entry j pools tokens stride*j .. stride*j + width - 1 and is rotated
  *   at position stride*j + pos_offset.  Entry j is visible to a query at

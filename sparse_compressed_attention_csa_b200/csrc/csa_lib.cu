@@ -114,8 +114,10 @@ csa_status_t check_dtype(csa_dtype_t dt) {
 }
 
 csa_status_t check_sizes(int B, int Tq, int n_max) {
-  if (B < 1 || Tq < 1 || n_max < 0 || B > 65535 || Tq > 65535)
-    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "B=%d Tq=%d n_max=%d out of range", B, Tq, n_max);
+  // query rows (B * Tq) index a grid dimension of at most 65535 blocks
+  if (B < 1 || Tq < 1 || n_max < 0 || (long long)B * Tq > 65535)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "B=%d Tq=%d n_max=%d out of range (B*Tq <= 65535)",
+                B, Tq, n_max);
   return CSA_OK;
 }
 

@@ -59,6 +59,17 @@ def _status(fn, *args):
     return ei.value.status
 
 
+def test_query_rows_beyond_one_grid_dimension_are_rejected(lib):
+    p = csa.Params()
+    assert csa.csa_workspace_size(p, csa.CSA_OP_SPARSE_ATTN, 255, 257, 100) >= 0  # 65535 rows
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_workspace_size(p, csa.CSA_OP_SPARSE_ATTN, 256, 257, 100)
+    assert ei.value.status == 3
+    with pytest.raises(csa.CsaError) as ei:
+        csa.csa_workspace_size(p, csa.CSA_OP_INDEX_TOPK, 0, 1, 100)
+    assert ei.value.status == 3
+
+
 def test_workspace_sizes(lib):
     p = csa.Params()
     n = csa.csa_workspace_size(p, csa.CSA_OP_INDEX_TOPK, 32, 1, 16383)

@@ -124,6 +124,19 @@ def test_decode_fewer_visible_than_k():
     check_decode(W.CSA_DECODE_64K.replace(B=2, T=2100, seed=22))  # N = 524 < 1024
 
 
+def test_decode_context_too_short_for_any_entry():
+    # T = 5 < width: no compressed entry, so no scores, every index -1 and the
+    # attention runs over the window and the sink only
+    check_decode(W.CSA_DECODE_64K.replace(B=2, T=5, seed=33))
+
+
+def test_decode_rows_at_the_tensor_core_cap_and_beyond():
+    # 1,900 selected + 128 window rows fill the tensor-core kernel's row list;
+    # 1,950 + 128 go past it and take the generic kernel
+    check_decode(W.CSA_DECODE_64K.replace(B=2, T=10000, topk=1900, seed=34))
+    check_decode(W.CSA_DECODE_64K.replace(B=2, T=10000, topk=1950, seed=35))
+
+
 def test_prefill_ragged_small():
     check_prefill(W.CSA_PREFILL_8K.replace(T=777, topk=64, seed=23))
 
