@@ -207,14 +207,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const int rope0 = kAtDim - a.rope_dim;
   // 128-dim chunks in streaming order: the others first, then the own ones
   // (own chunks: dims part * kOCols ..)
+  // (own chunks: dims part * kOCols ..).  Closed forms rather than small
+  // arrays: a run-time index would put them in local memory, and the MMA
+  // operands built from them would no longer be known to be warp-uniform.
   const int own0 = part * kOwn;
-  int chunk_of[4];
-  {
-    int w = 0;
-    for (int c = 0; c < 4; ++c)
-      if (c < own0 || c >= own0 + kOwn) chunk_of[w++] = c;
-    for (int c = 0; c < kOwn; ++c) chunk_of[w++] = own0 + c;
-  }
+  auto chunk_of = [&](int ck) {
+    return ck < 4 - kOwn ? (ck < own0 ? ck : ck + kOwn) : own0 + ck - (4 - kOwn);
+  };
   // q sub-block sb (64 dims) lives in shared memory (own half, NQ = 2) or in
   // TMEM at column 32 * q_tidx(sb); TMEM-bound sub-blocks are staged in the
   // last ring slots
@@ -298,10 +297,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const int i = k * 128 + tid;
         jv[k] = i < a.topk ? sel[i] : -1;
       }
-#pragma unroll
-      for (int k = 0; k < kMaxK; ++k) {
+#pragma unroll 1
+      for (int k = 0; k < kMaxK; ++k) {  // rolled: runs once per CTA (code size)
         if (k * 128 >= a.topk) break;
-        int j = jv[k];
+        int j = jv[0];
+#pragma unroll
+        for (int kk = 1; kk < kMaxK; ++kk) j = k == kk ? jv[kk] : j;
         if (j >= a.n_max) {
           report_error(CSA_ERR_DEVICE_BOUNDS);
           j = -1;
@@ -643,7 +644,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         }
       }
       for (int ck = 0; ck < 4; ++ck, ++n) {
-        const int chunk = chunk_of[ck];
+        const int chunk = chunk_of(ck);
         const int slot = n % kSlots;
         okp = mbar_wait(&sm.empty[slot], ((uint32_t)(n / kSlots) & 1u) ^ 1u, abortp);
         if (okp && !staged && slot >= kSlots - Lay::kQStage) {  // slot still holds q staging
@@ -668,7 +669,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     constexpr uint32_t id_qk = idesc_bf16_f32(128, kAtTile);
     constexpr uint32_t id_pv = idesc_bf16_f32(128, 128, 0, 1);
     int n = 0;  // chunks consumed
-    int own_slot[2][kOwn];
+    // ring slot of own chunk oc of tile j: chunk n = 4 j + ck goes to slot
+    // n % kSlots, and the own chunks are the last kOwn of a tile
+    auto own_slot = [&](int j, int oc) { return (4 * j + (4 - kOwn) + oc) % kSlots; };
     int last_pv = -1, last_s = -1;
     load_split();
     bool okm = rows_ok && mbar_wait(&sm.q_ready, 0, abortp);
@@ -681,14 +684,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 #pragma unroll
       for (int oc = 0; oc < kOwn; ++oc) {
         const uint64_t vd0 =
-            sw128_desc(smem_u32(ring + own_slot[sb][oc] * kAtChunkBytes), kAtChunkBytes / 2, 1024);
+            sw128_desc(smem_u32(ring + own_slot(j, oc) * kAtChunkBytes), kAtChunkBytes / 2, 1024);
 #pragma unroll
         for (int ks = 0; ks < kAtTile / 16; ++ks)
           mma_ts(t_o + (uint32_t)(oc * 128), t_s + (uint32_t)(sb * 64 + ks * 8),
                  vd0 + (uint64_t)((ks * 16 * 128) >> 4), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
       }
 #pragma unroll
-      for (int oc = 0; oc < kOwn; ++oc) tc_commit(&sm.empty[own_slot[sb][oc]]);
+      for (int oc = 0; oc < kOwn; ++oc) tc_commit(&sm.empty[own_slot(j, oc)]);
       tc_commit(&sm.pv_done[sb]);
       last_pv = j;
       return true;
@@ -705,10 +708,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
       // S(i) = Q K_i^T over the four 128-dim chunks (others first)
       for (int ck = 0; ck < 4 && okm; ++ck, ++n) {
-        const int chunk = chunk_of[ck];
+        const int chunk = chunk_of(ck);
         const bool own = ck >= 4 - kOwn;
         const int slot = n % kSlots;
-        if (own) own_slot[sb][ck - (4 - kOwn)] = slot;
         // wait for the chunk; meanwhile the previous tile's PV goes in as
         // soon as its P is ready (so that its V slots are released early)
         {
@@ -842,32 +844,36 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         okm = all != 0;
       }
       if (okm) {
+        // Rolled loops: this code runs once per CTA, so its size (instruction
+        // fetch) costs more than loop overhead.  The sum starts at -0, which
+        // adds exactly (x + -0 = x), so the first split enters unchanged.
 #pragma unroll 1
         for (int sl = s_lo; sl < s_hi; ++sl) {
           float o[32];
-          bool have = false;
-          int j = 0;
 #pragma unroll
-          for (int sp = 0; sp < kAtMaxSplits; ++sp) {
-            if (sp >= S) break;
+          for (int e = 0; e < 32; ++e) o[e] = -0.f;
+#pragma unroll 1
+          for (int sp = 0, j = 0; sp < S; ++sp) {
+            float wsp = mv[0];
+#pragma unroll
+            for (int k = 1; k < kAtMaxSplits; ++k) wsp = sp == k ? mv[k] : wsp;
             float tm[32];
             if (sp == split) {
-              own_slab(sl, lane_base, mv[sp], tm);
+              own_slab(sl, lane_base, wsp, tm);
             } else {
               const uint8_t* src = pbuf + (j * ns + (sl - s_lo)) * kAtSlabBytes;
 #pragma unroll
               for (int u = 0; u < 8; ++u) {
                 const float4 x = *reinterpret_cast<const float4*>(src + (u * kAtHeads + head) * 16);
-                tm[4 * u] = __fmul_rn(x.x, mv[sp]);
-                tm[4 * u + 1] = __fmul_rn(x.y, mv[sp]);
-                tm[4 * u + 2] = __fmul_rn(x.z, mv[sp]);
-                tm[4 * u + 3] = __fmul_rn(x.w, mv[sp]);
+                tm[4 * u] = __fmul_rn(x.x, wsp);
+                tm[4 * u + 1] = __fmul_rn(x.y, wsp);
+                tm[4 * u + 2] = __fmul_rn(x.z, wsp);
+                tm[4 * u + 3] = __fmul_rn(x.w, wsp);
               }
               ++j;
             }
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = have ? __fadd_rn(o[e], tm[e]) : tm[e];
-            have = true;
+            for (int e = 0; e < 32; ++e) o[e] = __fadd_rn(o[e], tm[e]);
           }
           out_slab(obuf, sl, sl - s_lo, o);
         }
