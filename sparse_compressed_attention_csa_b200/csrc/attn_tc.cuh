@@ -206,7 +206,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rope0 = kAtDim - a.rope_dim;
   // 128-dim chunks in streaming order: the others first, then the own ones
-  // (own chunks: dims part * kOCols ..)
   // (own chunks: dims part * kOCols ..).  Closed forms rather than small
   // arrays: a run-time index would put them in local memory, and the MMA
   // operands built from them would no longer be known to be warp-uniform.
