@@ -9,23 +9,23 @@
 // split over NQ CTAs by output dims: CTA `part` owns d_v columns
 // [part * 512/NQ, (part + 1) * 512/NQ) and computes S = Q K^T itself.
 //
-//   NQ = 2 (many queries: prefill; S recomputed twice)
+//   NQ = 2 (the one the library launches; S recomputed twice)
 //     TMEM  O [0,256) | S0 [256,320) | S1 [320,384) | Q other half [384,512)
 //     SMEM  Q own half (64 KB) | ring of 9 chunks | row list
-//   NQ = 4 (few queries: decode; S recomputed four times, but the whole of Q
-//           sits in TMEM, which frees shared memory for a deeper gather ring)
+//   NQ = 4 (the template supports it; measured slower on every workload:
+//           S recomputed four times, the whole of Q in TMEM, 13-chunk ring)
 //     TMEM  O [0,128) | S0 [128,192) | S1 [192,256) | Q [256,512)
 //     SMEM  ring of 13 chunks | row list
 //
 // Q is rotated at the query position and rounded to bf16 once, after one TMA
 // load of [128 heads][64 dims] boxes.  KV rows are gathered 64 at a time by
-// 128 threads with 16-byte cp.async into 128B-swizzled shared memory (the
-// gather reaches full bandwidth only with many requests in flight, which
-// many issuing threads sustain and one-warp TMA gathers do not).  A row
-// streams as four 128-dim chunks through a FIFO ring; chunks outside the
-// CTA's output dims feed only S and are released right after it, the CTA's
-// own chunks then serve as V for the PV product and are held until it
-// completes.  The row list holds selected entries, then window rows, each
+// 128 threads with 16-byte cp.async into 128B-swizzled shared memory (many
+// requests in flight from many issuing threads; a TMA row gather was not
+// built, since its 4-row destinations would sit at 512-byte offsets inside
+// the 1,024-byte swizzle atom).  A row streams as four 128-dim chunks
+// through a FIFO ring; chunks outside the CTA's output dims feed only S and
+// are released right after it, the CTA's own chunks then serve as V for the
+// PV product and are held until it completes.  The row list holds selected entries, then window rows, each
 // padded to a multiple of 4 with masked rows.
 //
 //   warp 8 (one thread): MMAs   S(i) = Q K_i^T  (N = 64, K = 512)

@@ -294,8 +294,8 @@ bool attn_tc_ok(const csa_params_t* p, csa_dtype_t dtype, bool hca, int n_max) {
 
 // Output-dim parts per query.  Two CTAs per query (q half in TMEM, half in
 // shared memory) measured faster than four (whole q in TMEM, deeper gather
-// ring, four-fold S recompute) on every workload here, so NQ = 4 is kept
-// compiled but not selected.
+// ring, four-fold S recompute) on every workload here, so only NQ = 2 is
+// instantiated.
 int attn_nq(int B, int Tq) { (void)B; (void)Tq; return 2; }
 
 // Clusters of `cluster` attention CTAs that fit on the device at once (0 if
@@ -720,7 +720,6 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   CSA_CHECK(make_tmap_bf16(&tq, g.q, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
   CSA_CHECK(make_tmap_bf16(&to, g.out, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 32, kAtHeads,
                            CU_TENSOR_MAP_SWIZZLE_64B));
-  if (attn_nq(g.B, g.Tq) == 4) return launch_attn_tc_nq<kHca, 4>(g, a, sp, ws, tq, to, s);
   return launch_attn_tc_nq<kHca, 2>(g, a, sp, ws, tq, to, s);
 }
 
