@@ -17,7 +17,7 @@ from sparse_compressed_attention_csa_b200 import (CSA_OP_SPARSE_ATTN, CSA_OP_TOP
                                                   CsaError, Params,
                                                   csa_compress, csa_workspace_size,
                                                   csa_index_scores, csa_poll_device_error,
-                                                  csa_sparse_attn, csa_topk_select, layer)
+                                                  csa_sparse_attn, csa_topk_select)
 from sparse_compressed_attention_csa_b200 import workloads as W
 from sparse_compressed_attention_csa_b200.workloads import bits_to_f32, to_f64
 

@@ -11,7 +11,6 @@ uses a caller workspace, and that sizes beyond the array are rejected.
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
 """
-import numpy as np
 import pytest
 import torch
 
