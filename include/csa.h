@@ -224,6 +224,15 @@ csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t dtype, co
                                     const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
                                     int32_t* idx_out, void* stream);
 
+/* Limit, in nanoseconds, of every bounded wait inside the library's kernels
+ * (a wait on a copy, an MMA or a cooperating CTA).  A wait that runs out
+ * records CSA_ERR_DEVICE_TIMEOUT (read with csa_poll_device_error) and its
+ * kernel winds down without finishing its output.  0 restores the default
+ * of 2 s.  Process-wide, read when a kernel is launched (a captured CUDA
+ * graph keeps the limit it was captured with).  A diagnostic: a tiny limit
+ * makes the timeout path run on purpose. */
+void csa_set_wait_limit_ns(uint64_t ns);
+
 /* Number of kernels this library has launched (or recorded into a stream
  * capture) in this process so far, on every device and host thread.  A
  * diagnostic: the difference across one call is that call's kernel count. */

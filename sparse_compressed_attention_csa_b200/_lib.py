@@ -98,6 +98,8 @@ def _load():
     lib.csa_poll_device_error.argtypes = [_P]
     lib.csa_launch_count.restype = ctypes.c_uint64
     lib.csa_launch_count.argtypes = []
+    lib.csa_set_wait_limit_ns.restype = None
+    lib.csa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
               "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error",
               "csa_index_topk_noalloc"):
@@ -270,6 +272,12 @@ def hca_attn(p: Params, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, 
 def csa_launch_count() -> int:
     """Kernels launched (or captured) by the library so far in this process."""
     return int(_load().csa_launch_count())
+
+
+def csa_set_wait_limit_ns(ns: int = 0):
+    """Limit of every bounded wait in the library's kernels (0: the 2 s
+    default).  Read at launch; a diagnostic for exercising the timeout path."""
+    _load().csa_set_wait_limit_ns(int(ns))
 
 
 def csa_poll_device_error(stream=None):

@@ -12,8 +12,8 @@
 #include <cstring>
 #include <mutex>
 
+#include "attn_pair.cuh"
 #include "attn_simt.cuh"
-#include "attn_tc.cuh"
 #include "common.cuh"
 #include "compress.cuh"
 #include "csa.h"
@@ -286,66 +286,22 @@ size_t topk_ws_bytes(const csa_params_t* p, int B, int Tq, int n_max) {
 
 // Tensor-core attention applies to the measured head shape in bf16.
 bool attn_tc_ok(const csa_params_t* p, csa_dtype_t dtype, bool hca, int n_max) {
-  if (dtype != CSA_BF16 || p->d != kAtDim || p->n_heads != kAtHeads) return false;
-  if (p->rope_dim > kAtMaxRope) return false;
+  if (dtype != CSA_BF16 || p->d != kApDim || p->n_heads != kApHeads) return false;
+  if (p->rope_dim > kApMaxRope) return false;
   const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
-  return rows + 8 <= kAtRowCap;
+  return rows + 8 <= kApRowCap;
 }
 
-// Output-dim parts per query.  Two CTAs per query (q half in TMEM, half in
-// shared memory) measured faster than four (whole q in TMEM, deeper gather
-// ring, four-fold S recompute) on every workload here, so only NQ = 2 is
-// instantiated.
-int attn_nq(int B, int Tq) { (void)B; (void)Tq; return 2; }
-
-// Clusters of `cluster` attention CTAs that fit on the device at once (0 if
-// the query fails, e.g. without a device).  Cached per (device, size).
-int attn_max_clusters(int cluster) {
-  static std::mutex mu;
-  static int cache[64][kAtMaxSplits + 1];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  std::lock_guard<std::mutex> lock(mu);
-  int& c = cache[dev][cluster];
-  if (c != 0) return c;
-  const size_t smem = AtLayout<2>::kBytes + 1024;
-  if (set_smem_attr(k_attn_tc<false, 2>, smem, "k_attn_tc") != CSA_OK) return 0;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)cluster, 1, 1);
-  cfg.blockDim = dim3(kAtThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = (unsigned)cluster;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, k_attn_tc<false, 2>, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  c = n > 0 ? n : -1;
-  return n;
-}
-
-// KV splits per query token: enough CTAs to cover the SMs, at least one
-// 64-row tile per split, at most one cluster's worth, and no more than lets
-// every cluster of the grid be resident at once (the splits of a token
-// meet at a cluster barrier).
+// KV splits per query token: each token is a pair of CTAs (one cluster),
+// and its splits are further pairs, merged by k_attn_merge.  Enough pairs to
+// cover the SMs once, at least one 64-row tile per split.
 int attn_splits(const csa_params_t* p, bool hca, int B, int Tq, int n_max) {
-  const long long units = (long long)B * Tq * attn_nq(B, Tq);
+  const long long pairs = (long long)B * Tq;
   const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
-  long long s = num_sms() / units;
-  const long long max_s = (rows + kAtTile - 1) / kAtTile;
+  long long s = num_sms() / (2 * pairs);
+  const long long max_s = (rows + kApTile - 1) / kApTile;
   if (s > max_s) s = max_s;
-  if (s > kAtMaxSplits) s = kAtMaxSplits;
-  while (s > 1) {
-    const int fit = attn_max_clusters((int)s);
-    if (fit <= 0 || units <= fit) break;  // unknown (no device): keep s
-    --s;
-  }
+  if (s > kApMaxSplits) s = kApMaxSplits;
   return s < 1 ? 1 : (int)s;
 }
 
@@ -354,10 +310,14 @@ size_t attn_ws_bytes(const csa_params_t* p, csa_dtype_t dtype, bool hca, int B, 
   if (!attn_tc_ok(p, dtype, hca, n_max)) return 0;
   const int sp = attn_splits(p, hca, B, Tq, n_max);
   if (sp == 1) return 0;
-  const size_t units = (size_t)B * Tq * sp * attn_nq(B, Tq);
-  return round_up(units * kAtHeads * (kAtDim / attn_nq(B, Tq)) * sizeof(float), 256) +
-         round_up(units * 2 * kAtHeads * sizeof(float), 256);
+  const size_t units = (size_t)B * Tq * sp * 2;  // (token, split, part)
+  return round_up(units * kApHeads * kApHalf * sizeof(float), 256) +
+         round_up(units * 2 * kApHeads * sizeof(float), 256);
 }
+
+// Limit of every bounded device-side wait (csa_set_wait_limit_ns).
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
 
 }  // namespace
 }  // namespace csa
@@ -384,6 +344,10 @@ CSA_API const char* csa_status_string(csa_status_t s) {
 }
 
 CSA_API const char* csa_last_error_detail(void) { return g_detail; }
+
+CSA_API void csa_set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns == 0 ? kDefaultWaitNs : (unsigned long long)ns, std::memory_order_relaxed);
+}
 
 CSA_API uint64_t csa_launch_count(void) {
   return g_launches.load(std::memory_order_relaxed);
@@ -663,26 +627,6 @@ static csa_status_t launch_attn_simt(const AttnArgs& a, csa_dtype_t dtype, cudaS
   return launched("k_attn_simt");
 }
 
-template <bool kHca, int NQ>
-static csa_status_t launch_attn_tc_nq(const AttnArgs& g, AttnTcArgs& a, int sp, void* ws,
-                                      const CUtensorMap& tq, const CUtensorMap& to,
-                                      cudaStream_t s) {
-  using Lay = AtLayout<NQ>;
-  if (sp > 1) {
-    // workspace: partial O | partial (m, l)
-    const size_t units = (size_t)g.B * g.Tq * sp * NQ;
-    const size_t o_bytes = round_up(units * kAtHeads * (kAtDim / NQ) * sizeof(float), 256);
-    a.part_o = (float*)ws;
-    a.part_ml = (float*)((char*)ws + o_bytes);
-  }
-  const size_t smem = Lay::kBytes + 1024;
-  CSA_CHECK(set_smem_attr(k_attn_tc<kHca, NQ>, smem, "k_attn_tc"));
-  dim3 grid((unsigned)(NQ * sp), (unsigned)(g.B * g.Tq));
-  const cudaError_t e = launch_ex(k_attn_tc<kHca, NQ>, grid, dim3(kAtThreads), smem, s, sp, a, tq, to);
-  if (e != cudaSuccess) return cuda_fail(e, "k_attn_tc");
-  return launched("k_attn_tc");
-}
-
 template <bool kHca>
 static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, void* ws,
                                    size_t ws_bytes, cudaStream_t s) {
@@ -691,7 +635,7 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   if (ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes, need %zu", ws_bytes, need);
   if (need > 0) CSA_CHECK(check_ptr(ws, "ws"));
-  AttnTcArgs a;
+  AttnPairArgs a;
   a.q = (const __nv_bfloat16*)g.q;
   a.q_pos = g.q_pos;
   a.kv_cmp = (const __nv_bfloat16*)g.kv_cmp;
@@ -711,16 +655,51 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   a.rope_dim = g.rope_dim;
   a.scale_log2 = g.scale * 1.4426950408889634f;
   a.splits = sp;
+  a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   a.out = (__nv_bfloat16*)g.out;
   a.part_o = nullptr;
   a.part_ml = nullptr;
-  for (int i = 0; i < kAtMaxRope / 2; ++i)
+  if (sp > 1) {
+    // workspace: partial O | partial (m, l)
+    const size_t units = (size_t)g.B * g.Tq * sp * 2;
+    const size_t o_bytes = round_up(units * kApHeads * kApHalf * sizeof(float), 256);
+    a.part_o = (float*)ws;
+    a.part_ml = (float*)((char*)ws + o_bytes);
+  }
+  for (int i = 0; i < kApMaxRope / 2; ++i)
     a.freq[i] = i < g.rope_dim / 2 ? std::pow(g.theta, -2.0 * i / (double)g.rope_dim) : 0.0;
-  CUtensorMap tq, to;
-  CSA_CHECK(make_tmap_bf16(&tq, g.q, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 64, kAtHeads));
-  CSA_CHECK(make_tmap_bf16(&to, g.out, kAtDim, (uint64_t)g.B * g.Tq * kAtHeads, 32, kAtHeads,
+  CUtensorMap tq, to, tc, tr;
+  CSA_CHECK(make_tmap_bf16(&tq, g.q, kApDim, (uint64_t)g.B * g.Tq * kApHeads, 64, kApHeads));
+  CSA_CHECK(make_tmap_bf16(&to, g.out, kApDim, (uint64_t)g.B * g.Tq * kApHeads, 32, kApHeads,
                            CU_TENSOR_MAP_SWIZZLE_64B));
-  return launch_attn_tc_nq<kHca, 2>(g, a, sp, ws, tq, to, s);
+  // row gathers (one-row boxes of 64 dims); a cache with no rows is never
+  // read, and its map is made over q instead
+  const uint64_t n_cmp_rows = (uint64_t)g.B * g.n_max, n_raw_rows = (uint64_t)g.B * g.raw_max;
+  const uint64_t n_q_rows = (uint64_t)g.B * g.Tq * kApHeads;
+  CSA_CHECK(make_tmap_bf16(&tc, n_cmp_rows ? g.kv_cmp : g.q, kApDim,
+                           n_cmp_rows ? n_cmp_rows : n_q_rows, 64, 1));
+  CSA_CHECK(make_tmap_bf16(&tr, n_raw_rows ? g.kv_raw : g.q, kApDim,
+                           n_raw_rows ? n_raw_rows : n_q_rows, 64, 1));
+  CSA_CHECK(set_smem_attr(k_attn_pair<kHca>, kApSmemBytes, "k_attn_pair"));
+  dim3 grid((unsigned)(2 * sp), (unsigned)(g.B * g.Tq));
+  cudaError_t e =
+      launch_ex(k_attn_pair<kHca>, grid, dim3(kApThreads), kApSmemBytes, s, 2, a, tq, to, tc, tr);
+  if (e != cudaSuccess) return cuda_fail(e, "k_attn_pair");
+  CSA_CHECK(launched("k_attn_pair"));
+  if (sp == 1) return CSA_OK;
+  AttnMergeArgs m;
+  m.part_o = a.part_o;
+  m.part_ml = a.part_ml;
+  m.sink = g.sink;
+  m.q_pos = g.q_pos;
+  m.splits = sp;
+  m.rope_dim = g.rope_dim;
+  m.out = a.out;
+  for (int i = 0; i < kApMaxRope / 2; ++i) m.freq[i] = a.freq[i];
+  e = launch_ex(k_attn_merge, dim3(2 * kApSlabs, (unsigned)(g.B * g.Tq)), dim3(kApHeads), 0, s, 1,
+                m);
+  if (e != cudaSuccess) return cuda_fail(e, "k_attn_merge");
+  return launched("k_attn_merge");
 }
 
 static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32_t* q_pos,

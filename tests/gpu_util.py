@@ -1,5 +1,8 @@
 """Helpers shared by the GPU tests: move generated inputs to the device,
 run the layer through the C-ABI binding, compare with the oracle."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -36,6 +39,10 @@ def assert_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = ""):
     err = float(np.max(np.abs(got - want))) if got.size else 0.0
     nrm = float(np.linalg.norm(want))
     rel = float(np.linalg.norm(got - want)) / nrm if nrm > 0 else err
+    log = os.environ.get("CSA_ERRLOG")  # optional record of every comparison's error
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"what": what, "dtype": dtype, "max_abs": err, "rel_l2": rel}) + "\n")
     assert err <= tol_abs and rel <= tol_rel, f"{what}: max-abs {err:.3e} rel-L2 {rel:.3e}"
     return err, rel
 
