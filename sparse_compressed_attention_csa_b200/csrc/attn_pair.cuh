@@ -17,25 +17,25 @@
 // so every KV row is gathered once (each CTA reads its own 512 bytes of it)
 // and Q K^T is computed once.  TMEM per CTA: O [0,256) | S0 [256,320) |
 // S1 [320,384) | Q[:, D_c] as bf16 pairs [384,512).  Shared memory: a ring
-// of 8 chunks of 64 rows x 128 dims (a tile's two chunks sit in adjacent
-// slots, so one N = 256 MMA covers the tile's PV), four 16 KB receive
+// of 10 chunks of 64 rows x 128 dims (a tile's two chunks sit in adjacent
+// slots, so one N = 256 MMA covers the tile's PV), three 16 KB receive
 // buffers for the partner's partial logits, the row list.  Distributed
-// shared memory moves only ~14 GB/s per SM (measured, st.async), so the
-// 16 KB of a tile take ~1.1 us: the dedicated exchange warps keep that off
-// the softmax's path.
+// shared memory moves only ~14 GB/s per SM each way (measured with
+// st.async; ~20 with bulk copies), so the 16 KB of a tile take ~1.1 us.
 //
-//   warp 6 (one thread): MMAs   S(i) = Q K_i^T (N = 64, K = 256, A from TMEM)
+//   warp 8 (one thread): MMAs   S(i) = Q K_i^T (N = 64, K = 256, A from TMEM)
 //                               O   += P(j) V(j) (N = 256, A = P from TMEM)
-//   warps 4-5: q by TMA, then the gather: TMA tile::gather4 (four rows x 64
-//              dims per instruction) of the CTA's half of each row into
-//              128B-swizzled chunks; warp 4 + c fetches chunk c of every tile
-//   warps 7-10: the row list, then one head per thread (= TMEM lane): this CTA's partial
-//              logits of each tile, rounded to fp16, out to the partner
-//              (st.async into its receive buffers) as soon as QK lands
-//   warps 0-3: one head per thread: the partner's partial logits in, online
-//              softmax in the log2 domain with a lazy rescale, P back into
-//              TMEM as bf16; epilogue with the sink, the inverse output
-//              rotation and a TMA store.
+//   warps 4-7: q by TMA, the row list, then the gather: TMA tile::gather4
+//              (four rows x 64 dims per instruction) of the CTA's half of
+//              each row into 128B-swizzled chunks.  A gather4 holds its
+//              warp for ~60 ns (one warp moves ~16 GB/s), so four warps
+//              issue: warp 4 + (2 (i % 2) + c) fetches chunk c of tile i.
+//   warps 0-3: one head per thread (= TMEM lane): this CTA's partial logits
+//              of each tile, rounded to fp16, out to the partner (st.async
+//              into its receive buffers), the partner's in; online softmax
+//              in the log2 domain with a lazy rescale, P back into TMEM as
+//              bf16; epilogue with the sink, the inverse output rotation
+//              and a TMA store.
 //
 // The pair swaps the scaled partial logits rounded to fp16; each CTA adds
 // its own fp32 partial to the partner's fp16 one (one rounding of 2^-11
@@ -65,18 +65,18 @@ constexpr int kApDim = 512;
 constexpr int kApHalf = 256;                         // dims per CTA of the pair
 constexpr int kApTile = 64;                          // KV rows per tile (QK N)
 constexpr int kApChunkBytes = kApTile * 128 * 2;     // 64 rows x 128 dims bf16
-constexpr int kApSlots = 8;                          // ring: 4 tiles of 2 chunks
+constexpr int kApSlots = 10;                         // ring: 5 tiles of 2 chunks
 constexpr int kApQSlot0 = kApSlots - 4;              // q staging: the last 4 slots
 constexpr int kApXBytes = kApHeads * kApTile * 2;    // fp16 partial logits of a tile
-constexpr int kApXBufs = 4;                          // receive buffers (see the exchange)
+constexpr int kApXBufs = 3;                          // receive buffers (see the exchange)
 constexpr int kApSubBytes = kApHeads * 128;          // q box: [128 heads][64 dims]
 constexpr int kApRowCap = 2048;                      // rows per query token
 constexpr int kApMaxRope = 128;                      // rotated dims supported
-constexpr int kApMaxSplits = 32;                     // split-KV parts per query token
-constexpr int kApSlabBytes = kApHeads * 32 * 4;      // 32 dims of fp32 O, 128 heads
+constexpr int kApMaxSplits = 8;                      // split-KV parts per query token
+constexpr int kApSlabBytes = kApHeads * 32 * 2;      // 32 dims of fp16 O, 128 heads
 constexpr int kApOutBoxBytes = kApHeads * 64;        // 32 dims of bf16 output, 128 heads
 constexpr int kApSlabs = kApHalf / 32;
-constexpr int kApThreads = 352;  // 11 warps
+constexpr int kApThreads = 288;  // 9 warps
 constexpr float kApRescaleLog2 = 8.0f;
 constexpr int kApXOff = kApSlots * kApChunkBytes;
 constexpr int kApMiscOff = kApXOff + kApXBufs * kApXBytes;
@@ -99,7 +99,7 @@ struct AttnPairArgs {
   int splits;
   unsigned long long wait_ns;  // limit of every bounded wait
   __nv_bfloat16* out;          // splits == 1
-  float* part_o;   // splits > 1: [B*Tq][splits][2][8 slabs][8 units][128][4] unnormalised O
+  __half* part_o;  // splits > 1: [B*Tq][splits][2][8 slabs][4 units][128][8] O / l, fp16
   float* part_ml;  // [B*Tq][splits][2][2][128]  (m, l) in the log2 domain
   double freq[kApMaxRope / 2];  // RoPE frequencies theta^(-2i/rope_dim)
 };
@@ -108,7 +108,7 @@ struct ApMisc {
   int rows[kApRowCap];  // gather row coordinates
   float cs[kApMaxRope / 2], sn[kApMaxRope / 2];
   uint64_t full[kApSlots], empty[kApSlots];
-  uint64_t s_full[2], p_full[2], pv_done[2], sent[2], xfull[kApXBufs];
+  uint64_t s_full[2], p_full[2], pv_done[2], xfull[kApXBufs];
   uint64_t q_tma, q_ready, rows_ready, rope_ready, mma_drain;
   uint32_t tmem_base;
   int n_rows;  // padded rows (multiple of 4)
@@ -116,13 +116,14 @@ struct ApMisc {
   int n_win;   // window rows (valid rows [pad4(n_sel), pad4(n_sel) + n_win))
   int abort_flag;
   int scan_tmp[4];
+  int last_n[kApSlots];  // last chunk requested into each ring slot (-1: none)
 };
 
 constexpr size_t kApSmemBytes = (size_t)kApMiscOff + sizeof(ApMisc) + 1024;
 static_assert(kApSmemBytes <= 232448, "shared memory budget");
 
 // The epilogue stages the output in the idle ring: 8 bf16 boxes of 8 KB
-// (one split), or the 8 fp32 slabs of 16 KB of the unnormalised O (splits).
+// (one split), or the 8 fp16 slabs of 8 KB of the split's O / l (splits).
 static_assert(kApSlabs * kApSlabBytes <= kApXOff, "epilogue staging fits the ring");
 
 // 2^x by the hardware approximation (relative error ~2^-22; the softmax
@@ -219,8 +220,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.p_full[i], 128);
       mbar_init(&sm.pv_done[i], 1);
-      mbar_init(&sm.sent[i], 128);
     }
+    for (int i = 0; i < kApSlots; ++i) sm.last_n[i] = -1;
     for (int i = 0; i < kApXBufs; ++i) mbar_init(&sm.xfull[i], 1);  // expect_tx + 16 KB in
     mbar_init(&sm.q_tma, 1);
     mbar_init(&sm.q_ready, 128);
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
     sm.abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 6) {
+  if (warp == 8) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
@@ -257,7 +258,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
     for (int sb = 0; sb < 4; ++sb)
       tma_load_2d(q_stage + sb * kApSubBytes, &tm_q, &sm.q_tma, dim0 + sb * 64, row_q * kApHeads);
   }
-  if (warp == 6) {
+  if (warp == 8) {
     // RoPE table at the query position
     for (int i = lane; i < a.rope_dim / 2; i += 32) {
       float c, s;
@@ -268,12 +269,12 @@ __global__ void __launch_bounds__(kApThreads, 1)
     mbar_arrive(&sm.rope_ready);
   }
 
-  if (warp >= 7) {
-    // ======================= row list (warps 7-10): gather coordinates of the
+  if (warp >= 4 && warp < 8) {
+    // ======================= row list (warps 4-7): gather coordinates of the
     // selected (or visible) entries in their order, then the window's raw
     // rows, each part padded to a multiple of 4 rows.  Both CTAs of a pair
     // build the same list.
-    const int tid = threadIdx.x - 224;
+    const int tid = threadIdx.x - 128;
     const int cmp_y0 = b * a.n_max;
     const int raw_y0 = b * a.raw_max;
     const int rp0 = a.raw_pos0[b];
@@ -308,13 +309,13 @@ __global__ void __launch_bounds__(kApThreads, 1)
         const int n = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += n;
       }
-      if (lane == 31) sm.scan_tmp[warp - 7] = x;
+      if (lane == 31) sm.scan_tmp[warp - 4] = x;
       asm volatile("bar.sync 2, 128;" ::: "memory");
       int off = x - cnt, tot = 0;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         const int c = sm.scan_tmp[w];
-        off += w < warp - 7 ? c : 0;
+        off += w < warp - 4 ? c : 0;
         tot += c;
       }
 #pragma unroll
@@ -415,9 +416,18 @@ __global__ void __launch_bounds__(kApThreads, 1)
       x_posted = min(ntile, kApXBufs);
       for (int i = 0; i < x_posted; ++i) mbar_arrive_expect_tx(&sm.xfull[i], kApXBytes);
     }
+    const uint32_t peer_x = mapa(xbuf, peer);  // the partner's receive buffers
+    const uint32_t peer_xfull = mapa(&sm.xfull[0], peer);
     const uint32_t xrow = (uint32_t)head * 128u;
 
     // ---- online softmax over the tiles
+    // Exchange: tile i's partial logits go to the partner's buffer i % 3.
+    // Three buffers need no handshake: before this CTA can send tile i + 3,
+    // its QK(i + 3) needs the PV of tile i + 1 issued, hence P(i + 1), hence
+    // the partner's tile i + 1, which the partner sends only after it has
+    // read tile i from that buffer (each thread reads tile i before it sends
+    // tile i + 1).  (Sending one tile ahead of the softmax instead measured
+    // slower: with two S buffers the next QK is not ready in time.)
     const int n_sel = sm.n_sel, ps = (n_sel + 3) & ~3, pe = ps + sm.n_win;
     for (int i = 0; i < ntile && ok; ++i) {
       const int sb = i & 1;
@@ -439,13 +449,26 @@ __global__ void __launch_bounds__(kApThreads, 1)
           z[32 + e] = __uint_as_float(rb[e]) * a.scale_log2;
         }
       }
-      // ---- the partner's tile i
+      // ---- out: fp16 pairs into the partner's buffer xb
+      {
+        const uint32_t dst = peer_x + (uint32_t)(xb * kApXBytes) + xrow;
+        const uint32_t bar = peer_xfull + (uint32_t)(xb * 8);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = make_uint4(ap_f16x2_sat(z[8 * u], z[8 * u + 1]),
+                                     ap_f16x2_sat(z[8 * u + 2], z[8 * u + 3]),
+                                     ap_f16x2_sat(z[8 * u + 4], z[8 * u + 5]),
+                                     ap_f16x2_sat(z[8 * u + 6], z[8 * u + 7]));
+          st_async_v4(dst + (uint32_t)((u ^ (head & 7)) << 4), v, bar);
+        }
+      }
+      // ---- in: the partner's tile i
       ok = __all_sync(0xffffffffu, mbar_wait_cluster(&sm.xfull[xb], (uint32_t)(i / kApXBufs) & 1u,
                                                      abortp, wait_ns));
       if (!ok) break;
       if (threadIdx.x == 0) {
         x_recv = i + 1;
-        if (i + kApXBufs < ntile) {  // the partner's tile i + 4 lands in this buffer next
+        if (i + kApXBufs < ntile) {  // the partner's tile i + 3 lands in this buffer next
           mbar_arrive_expect_tx(&sm.xfull[xb], kApXBytes);
           x_posted = i + kApXBufs + 1;
         }
@@ -529,10 +552,6 @@ __global__ void __launch_bounds__(kApThreads, 1)
         pk[e] = *reinterpret_cast<uint32_t*>(&pb);
       }
       l_run += ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
-      // P overwrites S(i): the exchange warps have read it
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(&sm.sent[sb], (uint32_t)(i >> 1) & 1u, abortp, wait_ns));
-      if (!ok) break;
       uint32_t w16[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) w16[e] = pk[e];
@@ -603,13 +622,15 @@ __global__ void __launch_bounds__(kApThreads, 1)
           bulk_wait_read_all();
         }
       } else {
-        // split-KV: this split's (m, l) and unnormalised O for k_attn_merge.
-        // O leaves through the ring as 8 contiguous 16 KB slabs
-        // ([16-byte unit u][head][4 floats] per 32 dims) and bulk copies.
+        // split-KV: this split's (m, l) and its O / l in fp16 for
+        // k_attn_merge (values of order one: fp16 keeps 11 bits).  O leaves
+        // through the ring as 8 contiguous 8 KB slabs ([16-byte unit u][head]
+        // [8 halves] per 32 dims) and one bulk copy.
         const size_t unit = ((size_t)row_q * S + split) * 2 + part;
         float* pml = a.part_ml + unit * 2 * kApHeads;
         pml[head] = m_run;
         pml[kApHeads + head] = l_run;
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
         for (int sl = 0; sl < kApSlabs; ++sl) {
           uint32_t r[32];
@@ -622,36 +643,39 @@ __global__ void __launch_bounds__(kApThreads, 1)
           }
           uint8_t* slab = ring + sl * kApSlabBytes;
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
+          for (int u = 0; u < 4; ++u) {
+            uint32_t h[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              h[k] = ap_f16x2_sat(__uint_as_float(r[8 * u + 2 * k]) * inv_l,
+                                  __uint_as_float(r[8 * u + 2 * k + 1]) * inv_l);
             *reinterpret_cast<uint4*>(slab + (u * kApHeads + head) * 16) =
-                make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+                make_uint4(h[0], h[1], h[2], h[3]);
+          }
         }
         fence_proxy_async_shared();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == 0) {
-          for (int sl = 0; sl < kApSlabs; ++sl)
-            bulk_store(a.part_o + unit * kApHeads * kApHalf + sl * (kApSlabBytes / 4),
-                       ring + sl * kApSlabBytes, kApSlabBytes);
+          bulk_store(a.part_o + unit * kApHeads * kApHalf, ring, kApSlabs * kApSlabBytes);
           bulk_commit();
           bulk_wait_read_all();
         }
       }
     }
-  } else if (warp < 6) {
-    // ======================= gather producers (warps 4-5)
+  } else if (warp < 8) {
+    // ======================= gather producers (warps 4-7)
     // Chunk n (tile n / 2, dims dim0 + 128 (n % 2)) goes to ring slot
-    // n % kApSlots; warp 4 + (n % 2) fetches it.  Lane l fetches rows
-    // 4 (l & 15) .. + 3 of the tile, 64-dim half l >> 4, with one gather4.
-    // Groups past the split end (only in its last tile) are zero-filled, so
-    // that masked rows hold finite values.
+    // n % kApSlots; warp 4 + (2 (i % 2) + c) fetches chunk c of tile i.
+    // Lane l fetches rows 4 (l & 15) .. + 3 of the tile, 64-dim half l >> 4,
+    // with one gather4.  Groups past the split end (only in its last tile)
+    // are zero-filled, so that masked rows hold finite values.
     load_split();
-    const int ck = warp - 4;
+    const int ck = (warp - 4) & 1, tpar = (warp - 4) >> 1;
     const int h = lane >> 4, rg = lane & 15;
     const int ps = (sm.n_sel + 3) & ~3;
     bool okp = __all_sync(0xffffffffu, rows_ok);
     bool staged = false;  // q staging slots handed back
-    int issued = 0;       // tiles whose chunk this warp has requested
-    for (int i = 0; i < ntile && okp; ++i) {
+    for (int i = tpar; i < ntile && okp; i += 2) {
       const int n = 2 * i + ck;
       const int slot = n % kApSlots;
       if (lane == 0) {
@@ -673,64 +697,15 @@ __global__ void __launch_bounds__(kApThreads, 1)
         fence_proxy_async_shared();  // read by the MMA (async proxy)
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)__popc(vmask) * 512u);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)__popc(vmask) * 512u);
+        sm.last_n[slot] = n;
+      }
       if (valid)
         tma_gather4(dst, g < ps ? &tm_cmp : &tm_raw, &sm.full[slot], dim0 + ck * 128 + h * 64,
                     sm.rows[g], sm.rows[g + 1], sm.rows[g + 2], sm.rows[g + 3]);
-      issued = i + 1;
     }
-    // every gather lands before the CTA may exit: the ring holds this warp's
-    // last kApSlots / 2 chunks at most (earlier slots were refilled, so their
-    // copies had landed)
-    if (lane == 0) {
-      int never = 0;
-      for (int i = max(0, issued - kApSlots / 2); i < issued; ++i) {
-        const int n = 2 * i + ck;
-        mbar_wait(&sm.full[n % kApSlots], (uint32_t)(n / kApSlots) & 1u, &never, kApDrainNs);
-      }
-    }
-  } else if (warp >= 7) {
-    // ======================= exchange warps (7-10, TMEM lane quarter warp % 4)
-    // Tile i's partial logits go to the partner's receive buffer i % 4.
-    // Four buffers need no handshake: this CTA's S(i) needs its PV(i - 2),
-    // hence its P(i - 2), hence the partner's tile i - 2, which the partner
-    // sends only after its QK(i - 2), after its PV(i - 4), after its P(i - 4):
-    // the partner has read tile i - 4 from the buffer before tile i can come.
-    const int head = (warp & 3) * 32 + lane;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    load_split();
-    bool okx = __all_sync(0xffffffffu, rows_ok);
-    const uint32_t peer_x = mapa(xbuf, peer);
-    const uint32_t peer_xfull = mapa(&sm.xfull[0], peer);
-    const uint32_t xrow = (uint32_t)head * 128u;
-    for (int i = 0; i < ntile && okx; ++i) {
-      const int sb = i & 1;
-      const int xb = i % kApXBufs;
-      okx = __all_sync(0xffffffffu,
-                       mbar_wait(&sm.s_full[sb], (uint32_t)(i >> 1) & 1u, abortp, wait_ns));
-      if (!okx) break;
-      tc_fence_after();
-      uint32_t ra[32], rb[32];
-      tmem_ld32(t_s + lane_base + (uint32_t)(sb * 64), ra);
-      tmem_ld32(t_s + lane_base + (uint32_t)(sb * 64 + 32), rb);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&sm.sent[sb]);  // S(i) read: the softmax may write P(i) over it
-      const uint32_t dst = peer_x + (uint32_t)(xb * kApXBytes) + xrow;
-      const uint32_t bar = peer_xfull + (uint32_t)(xb * 8);
-      const float sc = a.scale_log2;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t* r = u < 4 ? &ra[8 * u] : &rb[8 * (u - 4)];
-        const uint4 v = make_uint4(
-            ap_f16x2_sat(__uint_as_float(r[0]) * sc, __uint_as_float(r[1]) * sc),
-            ap_f16x2_sat(__uint_as_float(r[2]) * sc, __uint_as_float(r[3]) * sc),
-            ap_f16x2_sat(__uint_as_float(r[4]) * sc, __uint_as_float(r[5]) * sc),
-            ap_f16x2_sat(__uint_as_float(r[6]) * sc, __uint_as_float(r[7]) * sc));
-        st_async_v4(dst + (uint32_t)((u ^ (head & 7)) << 4), v, bar);
-      }
-    }
-  } else if (warp == 6 && lane == 0) {
+  } else if (warp == 8 && lane == 0) {
     // ======================= MMA issuer
     constexpr uint32_t id_qk = idesc_bf16_f32(128, kApTile);
     constexpr uint32_t id_pv = idesc_bf16_f32(128, kApHalf, 0, 1);
@@ -833,12 +808,19 @@ __global__ void __launch_bounds__(kApThreads, 1)
                         kApDrainNs);
   }
   if (warp == 4 && lane == 0) {
+    // every copy into shared memory lands before the CTA may exit: q, and in
+    // each ring slot the last chunk requested into it (an earlier one was
+    // consumed before the slot could be refilled)
     int never = 0;
     mbar_wait(&sm.q_tma, 0, &never, kApDrainNs);
+    for (int s = 0; s < kApSlots; ++s) {
+      const int n = sm.last_n[s];
+      if (n >= 0) mbar_wait(&sm.full[s], (uint32_t)(n / kApSlots) & 1u, &never, kApDrainNs);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 6) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -846,13 +828,13 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Split-KV merge: one CTA per (token, part, 32-dim slab), one head per
-// thread.  With the splits' (m_s, l_s) and unnormalised O_s of the head:
+// thread.  With the splits' (m_s, l_s) and normalised Ô_s = O_s / l_s:
 //   M = max(sink, max_s m_s),  L = 2^(sink - M) + sum_s l_s 2^(m_s - M)
-//   o = sum_s (2^(m_s - M) / L) O_s       (split order, products and sums
+//   o = sum_s (l_s 2^(m_s - M) / L) Ô_s   (split order, products and sums
 //                                          rounded one by one: deterministic)
 // then the RoPE dims rotated back by -t, bf16.
 struct AttnMergeArgs {
-  const float* part_o;
+  const __half* part_o;
   const float* part_ml;
   const float* sink;
   const int* q_pos;
@@ -882,37 +864,70 @@ __global__ void __launch_bounds__(kApHeads) k_attn_merge(AttnMergeArgs a) {
       sn[head] = s;
     }
   }
+  const size_t unit0 = (size_t)row_q * S * 2 + part;  // unit of split s: unit0 + 2 s
+  auto slab_of = [&](int s) {
+    return reinterpret_cast<const uint4*>(a.part_o + (unit0 + 2 * (size_t)s) * kApHeads * kApHalf) +
+           (size_t)sl * (kApSlabBytes / 16);
+  };
+  // every split's (m, l) and the first four splits' data, all in flight at once
+  float mv[kApMaxSplits], lv[kApMaxSplits];
+  uint4 x[4][4];
+#pragma unroll
+  for (int s = 0; s < kApMaxSplits; ++s) {
+    mv[s] = -INFINITY;
+    lv[s] = 0.f;
+    if (s < S) {
+      const float* ml = a.part_ml + (unit0 + 2 * s) * 2 * kApHeads;
+      mv[s] = __ldcg(ml + head);
+      lv[s] = __ldcg(ml + kApHeads + head);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      x[j][u] = j < S ? __ldcg(slab_of(j) + u * kApHeads + head) : make_uint4(0u, 0u, 0u, 0u);
   const float sink_l2 = a.sink[head] * 1.4426950408889634f;
   float M = sink_l2;
-  for (int s = 0; s < S; ++s) {
-    const size_t unit = ((size_t)row_q * S + s) * 2 + part;
-    M = fmaxf(M, __ldcg(a.part_ml + unit * 2 * kApHeads + head));
-  }
+#pragma unroll
+  for (int s = 0; s < kApMaxSplits; ++s) M = fmaxf(M, mv[s]);
   float L = exp2f(sink_l2 - M);
-  for (int s = 0; s < S; ++s) {
-    const size_t unit = ((size_t)row_q * S + s) * 2 + part;
-    const float m = __ldcg(a.part_ml + unit * 2 * kApHeads + head);
-    const float l = __ldcg(a.part_ml + unit * 2 * kApHeads + kApHeads + head);
-    if (m != -INFINITY) L += l * exp2f(m - M);
+#pragma unroll
+  for (int s = 0; s < kApMaxSplits; ++s) {
+    mv[s] = mv[s] == -INFINITY ? 0.f : lv[s] * exp2f(mv[s] - M);  // l_s 2^(m_s - M)
+    L += mv[s];
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   float o[32];
 #pragma unroll
   for (int e = 0; e < 32; ++e) o[e] = -0.f;  // x + -0 = x: the first split enters unchanged
-  for (int s = 0; s < S; ++s) {
-    const size_t unit = ((size_t)row_q * S + s) * 2 + part;
-    const float m = __ldcg(a.part_ml + unit * 2 * kApHeads + head);
-    const float w = m == -INFINITY ? 0.f : exp2f(m - M) * inv;
-    const float4* src = reinterpret_cast<const float4*>(
-        a.part_o + unit * kApHeads * kApHalf + (size_t)sl * (kApSlabBytes / 4));
+  auto accumulate = [&](const uint4 (&v)[4], float w) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 x = __ldcg(src + u * kApHeads + head);
-      o[4 * u] = __fadd_rn(o[4 * u], __fmul_rn(x.x, w));
-      o[4 * u + 1] = __fadd_rn(o[4 * u + 1], __fmul_rn(x.y, w));
-      o[4 * u + 2] = __fadd_rn(o[4 * u + 2], __fmul_rn(x.z, w));
-      o[4 * u + 3] = __fadd_rn(o[4 * u + 3], __fmul_rn(x.w, w));
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t hv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = ap_f16x2_to_f32(hv[k]);
+        o[8 * u + 2 * k] = __fadd_rn(o[8 * u + 2 * k], __fmul_rn(f.x, w));
+        o[8 * u + 2 * k + 1] = __fadd_rn(o[8 * u + 2 * k + 1], __fmul_rn(f.y, w));
+      }
     }
+  };
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (j < S) accumulate(x[j], mv[j] * inv);
+#pragma unroll
+  for (int s0 = 4; s0 < kApMaxSplits; s0 += 4) {
+    if (s0 >= S) break;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        x[j][u] = s0 + j < S ? __ldcg(slab_of(s0 + j) + u * kApHeads + head)
+                             : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (s0 + j < S) accumulate(x[j], mv[s0 + j] * inv);
   }
   if (rot) {
     __syncthreads();

@@ -294,12 +294,14 @@ bool attn_tc_ok(const csa_params_t* p, csa_dtype_t dtype, bool hca, int n_max) {
 
 // KV splits per query token: each token is a pair of CTAs (one cluster),
 // and its splits are further pairs, merged by k_attn_merge.  Enough pairs to
-// cover the SMs once, at least one 64-row tile per split.
+// cover the SMs once, at least two 64-row tiles per split (a split's fixed
+// costs - q, the row list, writing 128 KB of partial O - want rows to
+// spread over), at most kApMaxSplits.
 int attn_splits(const csa_params_t* p, bool hca, int B, int Tq, int n_max) {
   const long long pairs = (long long)B * Tq;
   const long long rows = (long long)(hca ? n_max : p->topk) + p->window;
   long long s = num_sms() / (2 * pairs);
-  const long long max_s = (rows + kApTile - 1) / kApTile;
+  const long long max_s = (rows + 2 * kApTile - 1) / (2 * kApTile);
   if (s > max_s) s = max_s;
   if (s > kApMaxSplits) s = kApMaxSplits;
   return s < 1 ? 1 : (int)s;
@@ -311,7 +313,7 @@ size_t attn_ws_bytes(const csa_params_t* p, csa_dtype_t dtype, bool hca, int B, 
   const int sp = attn_splits(p, hca, B, Tq, n_max);
   if (sp == 1) return 0;
   const size_t units = (size_t)B * Tq * sp * 2;  // (token, split, part)
-  return round_up(units * kApHeads * kApHalf * sizeof(float), 256) +
+  return round_up(units * kApHeads * kApHalf * sizeof(__half), 256) +
          round_up(units * 2 * kApHeads * sizeof(float), 256);
 }
 
@@ -423,7 +425,7 @@ static csa_status_t launch_index_tc(const void* q_idx, const float* w, const voi
   dim3 grid((unsigned)(qblocks * chunks), (unsigned)B);
   const cudaError_t e = launch_ex(k_index_scores_tc<QPB, STAGES>, grid, dim3(kIdxTcThreads), smem,
                                   s, 1, tk, tq, w, q_pos, n_cmp, Tq, n_max, width, stride, chunks,
-                                  scores);
+                                  g_wait_ns.load(std::memory_order_relaxed), scores);
   if (e != cudaSuccess) return cuda_fail(e, "k_index_scores_tc");
   return launched("k_index_scores_tc");
 }
@@ -662,8 +664,8 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   if (sp > 1) {
     // workspace: partial O | partial (m, l)
     const size_t units = (size_t)g.B * g.Tq * sp * 2;
-    const size_t o_bytes = round_up(units * kApHeads * kApHalf * sizeof(float), 256);
-    a.part_o = (float*)ws;
+    const size_t o_bytes = round_up(units * kApHeads * kApHalf * sizeof(__half), 256);
+    a.part_o = (__half*)ws;
     a.part_ml = (float*)((char*)ws + o_bytes);
   }
   for (int i = 0; i < kApMaxRope / 2; ++i)
