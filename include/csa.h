@@ -208,14 +208,17 @@ csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const void* q,
  * buffers, an engine whose allocator has already reserved all device
  * memory, or a latency-critical loop that cannot afford cudaMalloc's
  * device-wide synchronization.
- *   Scratch: a fixed array of 2^21 fp32 scores (8 MiB) compiled into the
- *   library; every GPU that loads the library holds it until the process
- *   exits.  B * Tq * n_max above 2^21 returns CSA_ERR_UNSUPPORTED_SHAPE.
- *   Nothing in the array needs clearing: each call writes every score it
- *   reads.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) and caches it; make that first call before any
- *   stream capture.
+ *   Scratch: a fixed 8 MiB array compiled into the library; every GPU that
+ *   loads the library holds it until the process exits.  It holds the
+ *   scores (B * Tq * n_max fp32, rounded up to 256 bytes) and, for rows too
+ *   long for one top-k block, the per-chunk candidate lists: the call needs
+ *   csa_workspace_size(CSA_OP_INDEX_TOPK) <= 8 MiB (so at most 2^21 scores)
+ *   and returns CSA_ERR_UNSUPPORTED_SHAPE beyond that.  Nothing in the array
+ *   needs clearing: each call writes everything it reads.
+ *   The first call in a CUDA context looks up the array's device address
+ *   (cudaGetSymbolAddress) and caches it under that context's id (a reset
+ *   device, or another context made current on the same device, looks it up
+ *   again); make that first call before any stream capture.
  *   Every call shares the one array: calls whose work overlaps on the GPU
  *   (different streams, or other host threads) race and give wrong indices.
  *   Serialize them. */

@@ -761,25 +761,62 @@ CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const vo
 constexpr size_t kNoAllocScoreFloats = size_t(1) << 21;  // B * Tq * n_max limit
 static __device__ __align__(256) float g_noalloc_scores[kNoAllocScoreFloats];
 
-// Device address of g_noalloc_scores on the current device.  In host code
+// Device address of g_noalloc_scores in the current context.  In host code
 // the symbol's name is only a host-side stand-in, so the address is looked
-// up with cudaGetSymbolAddress once per device (the first call on a device)
-// and cached.
-static csa_status_t noalloc_scores_ptr(float** out) {
-  static float* ptrs[64];
-  static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(CSA_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scores);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
-    ptrs[dev] = static_cast<float*>(p);
+// up with cudaGetSymbolAddress on the first call in a context and cached
+// under that context's unique id (a reset device or another context on the
+// same device loads the module again, possibly elsewhere, and gets its own
+// entry).
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+static csa_status_t current_context_id(unsigned long long* id) {
+  static PfnCtxGetCurrent get_current = nullptr;
+  static PfnCtxGetId get_id = nullptr;
+  if (get_current == nullptr || get_id == nullptr) {
+    void* p1 = nullptr;
+    void* p2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      return fail(CSA_ERR_CUDA, "driver entry points cuCtxGetCurrent / cuCtxGetId unavailable");
+    get_current = reinterpret_cast<PfnCtxGetCurrent>(p1);
+    get_id = reinterpret_cast<PfnCtxGetId>(p2);
   }
-  *out = ptrs[dev];
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+    return fail(CSA_ERR_CUDA, "no current CUDA context");
+  if (get_id(ctx, id) != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "cuCtxGetId failed");
+  return CSA_OK;
+}
+
+static csa_status_t noalloc_scores_ptr(float** out) {
+  struct Entry {
+    unsigned long long ctx;
+    float* ptr;
+  };
+  static Entry cache[64];
+  static int n_cache = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx) == CSA_OK;
+  if (have_ctx)
+    for (int i = 0; i < n_cache; ++i)
+      if (cache[i].ctx == ctx) {
+        *out = cache[i].ptr;
+        return CSA_OK;
+      }
+  // first call in this context (or none is current yet: the runtime makes
+  // the device's primary context current here)
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scores);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+  if (!have_ctx) CSA_CHECK(current_context_id(&ctx));
+  cache[n_cache < 64 ? n_cache++ : 63] = Entry{ctx, static_cast<float*>(p)};
+  *out = static_cast<float*>(p);
   return CSA_OK;
 }
 
@@ -804,9 +841,9 @@ CSA_API csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t d
   const size_t tb = topk_ws_bytes(p, B, Tq, n_max);
   if (sb + tb > kNoAllocScoreFloats * sizeof(float))
     return fail(CSA_ERR_UNSUPPORTED_SHAPE,
-                "B*Tq*n_max = %zu scores exceed the no-alloc scratch of %zu; use csa_index_topk "
-                "with a workspace",
-                (size_t)B * (size_t)Tq * (size_t)n_max, kNoAllocScoreFloats);
+                "scores (%zu bytes) and top-k candidate lists (%zu bytes) exceed the no-alloc "
+                "scratch of %zu bytes; use csa_index_topk with a workspace",
+                sb, tb, kNoAllocScoreFloats * sizeof(float));
   CSA_CHECK(check_device());
   float* scores = nullptr;
   CSA_CHECK(noalloc_scores_ptr(&scores));

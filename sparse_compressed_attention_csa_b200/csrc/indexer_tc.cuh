@@ -51,7 +51,8 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
     k_index_scores_tc(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_q, const float* __restrict__ w,
                       const int* __restrict__ q_pos, const int* __restrict__ n_cmp, int Tq,
-                      int n_max, int width, int stride, int chunks, float* __restrict__ scores) {
+                      int n_max, int width, int stride, int chunks, unsigned long long wait_ns,
+                      float* __restrict__ scores) {
   using namespace sm100;
   using S = IdxTcSmem<QPB, STAGES>;
   constexpr int N = S::kN;
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
       for (int i = 0; i < ntile; ++i) {
         const int s = i % STAGES;
         const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-        if (!mbar_wait(&sm.empty[s], ph ^ 1u, abortp)) break;
+        if (!mbar_wait(&sm.empty[s], ph ^ 1u, abortp, wait_ns)) break;
         mbar_arrive_expect_tx(&sm.full[s], S::kKBytes);
         const int row = b * n_max + (tb + i) * kIdxTcKeys;
         tma_load_2d(sm.keys[s], &tm_k, &sm.full[s], 0, row);
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, N);
       int last = -1;
-      if (mbar_wait(&sm.q_bar, 0, abortp)) {
+      if (mbar_wait(&sm.q_bar, 0, abortp, wait_ns)) {
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm.q);
         for (int i = 0; i < ntile; ++i) {
@@ -146,8 +147,8 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
           const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
           const int a = i & 1;
           const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-          if (!mbar_wait(&sm.acc_empty[a], aph ^ 1u, abortp)) break;
-          if (!mbar_wait(&sm.full[s], ph, abortp)) break;
+          if (!mbar_wait(&sm.acc_empty[a], aph ^ 1u, abortp, wait_ns)) break;
+          if (!mbar_wait(&sm.full[s], ph, abortp, wait_ns)) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(sm.keys[s]);
 #pragma unroll
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
     for (int i = 0; i < ntile; ++i) {
       const int a = i & 1;
       const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-      bool ok = mbar_wait(&sm.acc_full[a], aph, abortp);
+      bool ok = mbar_wait(&sm.acc_full[a], aph, abortp, wait_ns);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       float sc[QPB];

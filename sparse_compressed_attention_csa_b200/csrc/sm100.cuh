@@ -57,16 +57,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, suspending the thread for at most `hint_ns` while the
+// phase is incomplete.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity,
+                                                  uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint32_t suspend_hint(uint64_t limit_ns) {
+  return limit_ns < 0xFFFFFFFFull ? (uint32_t)limit_ns : 0xFFFFFFFFu;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false when
 // the CTA is aborting (flag set by another thread) or when this wait ran out
-// (then it sets the flag and records the timeout).
+// (then it sets the flag and records the timeout).  The clock is read after
+// the second unsuccessful try and every 64 tries, and no try suspends longer
+// than the limit, so even a limit of a few nanoseconds runs out on a phase
+// that is not complete at once.
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                        uint64_t limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = suspend_hint(limit_ns);
+  if (mbar_try_wait_for(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
+    if (mbar_try_wait_for(bar, parity, hint)) return true;
+    if ((it & 63u) == 1u) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
@@ -219,14 +242,15 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
                : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                      uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -236,11 +260,12 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
                                                volatile int* abort_flag,
                                                uint64_t limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint32_t hint = suspend_hint(limit_ns);
+  if (mbar_try_wait_cluster(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
+    if (mbar_try_wait_cluster(bar, parity, hint)) return true;
+    if ((it & 63u) == 1u) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;

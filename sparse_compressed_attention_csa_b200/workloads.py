@@ -150,8 +150,9 @@ def _ints(rng: np.random.Generator, shape, r: int, bf16: bool) -> np.ndarray:
     return out.reshape(shape)
 
 
-def generate(wl: Workload) -> dict:
-    """Draw every input of `wl`.
+def generate(wl: Workload, keys=None) -> dict:
+    """Draw every input of `wl` (or only those named in `keys`: each tensor
+    has its own stream, so skipping one changes no other).
 
     Returned keys (shapes; bf16 workloads give uint16 bit patterns for the
     big tensors, fp32 elsewhere):
@@ -167,16 +168,24 @@ def generate(wl: Workload) -> dict:
     st = _Streams(wl.seed)
     B, T, d, N, Tq = wl.B, wl.T, wl.d, wl.n_cmp, wl.Tq
     out: dict = {}
+    want = (lambda k: True) if keys is None else (lambda k: k in keys)
+
+    def normal(rng, shape, key):  # drawn only when wanted
+        return _normal(rng, shape, bf16) if want(key) else None
+
+    def ints(rng, shape, key):
+        return _ints(rng, shape, wl.int_range, bf16) if want(key) else None
+
     if wl.kind == "csa_prefill":
-        out["x"] = _normal(st["x"], (B, T, d), bf16)
-        out["g"] = _normal(st["g"], (B, T, d), bf16)
+        out["x"] = normal(st["x"], (B, T, d), "x")
+        out["g"] = normal(st["g"], (B, T, d), "g")
     if wl.kind in ("csa_prefill", "csa_decode"):
-        out["k_idx"] = _ints(st["k_idx"], (B, N, wl.idx_dim), wl.int_range, bf16)
-        out["q_idx"] = _ints(st["q_idx"], (B, Tq, wl.idx_heads, wl.idx_dim), wl.int_range, bf16)
+        out["k_idx"] = ints(st["k_idx"], (B, N, wl.idx_dim), "k_idx")
+        out["q_idx"] = ints(st["q_idx"], (B, Tq, wl.idx_heads, wl.idx_dim), "q_idx")
         e = st["w"].integers(0, len(wl.w_exps), size=(B, Tq, wl.idx_heads))
         out["w"] = np.exp2(np.asarray(wl.w_exps, dtype=np.float32)[e]).astype(np.float32)
         out["n_cmp"] = np.full((B,), N, dtype=np.int32)
-    out["q"] = _normal(st["q"], (B, Tq, wl.n_heads, d), bf16)
+    out["q"] = normal(st["q"], (B, Tq, wl.n_heads, d), "q")
     out["sink"] = st["sink"].standard_normal(wl.n_heads, dtype=np.float32)
     if wl.kind == "csa_prefill":
         out["q_pos"] = np.tile(np.arange(T, dtype=np.int32), (B, 1))
@@ -184,16 +193,11 @@ def generate(wl: Workload) -> dict:
         out["n_raw"] = np.full((B,), T, dtype=np.int32)
     else:
         out["q_pos"] = np.full((B, 1), T - 1, dtype=np.int32)
-        out["kv_cmp"] = _normal(st["kv_cmp"], (B, N, d), bf16)
+        out["kv_cmp"] = normal(st["kv_cmp"], (B, N, d), "kv_cmp")
         W = wl.window
-        out["kv_raw"] = _normal(st["kv_raw"], (B, W, d), bf16)
+        out["kv_raw"] = normal(st["kv_raw"], (B, W, d), "kv_raw")
         out["raw_pos0"] = np.full((B,), T - W, dtype=np.int32)
         out["n_raw"] = np.full((B,), W, dtype=np.int32)
         if wl.kind == "hca_decode":
             out["n_cmp"] = np.full((B,), N, dtype=np.int32)
-    return out
-
-
-def scaled(wl: Workload, **kw) -> Workload:
-    """A smaller (or otherwise changed) copy of a workload for parity runs."""
-    return wl.replace(**kw)
+    return {k: v for k, v in out.items() if v is not None}

@@ -6,7 +6,9 @@ engines whose allocator already owns all device memory, loops that cannot
 afford cudaMalloc's device-wide synchronization).  It keeps its scores in a
 fixed array built into the library.  This test checks, through the C ABI,
 that two calls in a row give exactly the indices of csa_index_topk, which
-uses a caller workspace, and that sizes beyond the array are rejected.
+uses a caller workspace (also for rows long enough to need the top-k
+candidate lists kept in the array), and that sizes beyond the array are
+rejected.
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
@@ -23,9 +25,12 @@ from sparse_compressed_attention_csa_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
+_KEYS = ("q_idx", "w", "k_idx", "q_pos", "n_cmp")
+
+
 def _inputs(wl):
-    d = W.generate(wl)
-    return {k: dev(d[k]) for k in ("q_idx", "w", "k_idx", "q_pos", "n_cmp")}
+    d = W.generate(wl, keys=_KEYS)
+    return {k: dev(d[k]) for k in _KEYS}
 
 
 def _with_workspace(p, t):
@@ -61,6 +66,20 @@ def test_no_alloc_matches_workspace_call_twice_in_a_row():
         assert int((got >= 0).sum()) > 0
 
 
+def test_no_alloc_long_rows_use_candidate_lists_from_its_array():
+    # 2 rows of 200,000 entries: too long for one top-k block, so each row is
+    # cut into chunks whose candidate lists sit in the array after the scores
+    wl = W.CSA_DECODE_1M.replace(B=2, T=4 * 200000 + 4, seed=43)
+    p = params_of(wl)
+    t = _inputs(wl)
+    want = _with_workspace(p, t)
+    got = _no_alloc(p, t)
+    torch.cuda.synchronize()
+    csa_poll_device_error()
+    assert torch.equal(got, want)
+    assert int((got >= 0).sum()) == 2 * p.topk
+
+
 def test_no_alloc_rejects_sizes_beyond_its_array():
     wl = W.CSA_DECODE_64K.replace(B=2, T=4 * 4096 + 4)   # small real inputs
     p = params_of(wl)
@@ -71,4 +90,4 @@ def test_no_alloc_rejects_sizes_beyond_its_array():
     with pytest.raises(CsaError) as ei:
         csa_index_topk_noalloc(p, t["q_idx"], t["w"], k_big, t["q_pos"], t["n_cmp"], idx)
     assert ei.value.status == 3
-    assert "no-alloc scratch" in str(ei.value)
+    assert "no-alloc scratch" in str(ei.value) and "bytes" in str(ei.value)
