@@ -37,6 +37,8 @@ Readings of points the pages leave open:
   sit at their own token position;
 * RoPE pairs are interleaved (d-r+2i, d-r+2i+1) with frequency
   theta**(-2i/r), rotated as a complex number times exp(i * pos * freq);
+  where a layer extends it with YaRN (theta = 160,000, factor 16 over
+  65,536 tokens), one YaRN spec serves q, entries, window rows and output;
 * the softmax scale is 1/sqrt(d) on the whole q.k; the sink logit is not
   scaled;
 * entry j is visible to the query at token t iff its last token
@@ -51,6 +53,9 @@ path as parameters): entry position, RoPE pair layout, window inclusivity,
 decode query position.
 """
 from __future__ import annotations
+
+import math
+from dataclasses import dataclass
 
 import numpy as np
 
@@ -86,12 +91,60 @@ def window_tokens(t: int, window: int, raw_pos0: int, n_raw: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Extended RoPE of the compressed layers ("DeepSeek-V4-Pro vs Inkling" and
+# "DeepSeek-V4.1-Flash vs Inkling", "Partial RoPE" rows: theta = 160,000
+# with YaRN, factor 16 over 65,536 tokens; "DeepSeek-V4-Pro" fact sheet,
+# raw config field compress_rope_theta 160000).  The pages give no YaRN
+# formula; this follows the published definition (Peng, Quesnelle, Fan,
+# Shippole 2023, "YaRN: Efficient Context Window Extension of Large Language
+# Models", section 3): per rotary pair i with frequency f_i = theta**(-2i/r)
+# and wavelength 2 pi / f_i, r_i = L / wavelength counts the rotations the
+# pair makes over the original context L; with
+#   gamma_i = clip((r_i - alpha) / (beta - alpha), 0, 1)
+# the new frequency is (1 - gamma_i) f_i / s + gamma_i f_i (pairs that turn
+# fewer than alpha times are interpolated by the factor s, pairs that turn
+# more than beta times keep their frequency), and the softmax logits are
+# multiplied by (0.1 ln s + 1)**2 (the paper's attention temperature).
+# alpha = 1 and beta = 32 are the paper's values.
+# --------------------------------------------------------------------------
+@dataclass(frozen=True)
+class YaRN:
+    theta: float            # RoPE base
+    factor: float           # s, the context-extension factor
+    orig_ctx: int           # L, the context the frequencies were made for
+    beta_fast: float = 32.0  # beta: rotations over L above which f_i is kept
+    beta_slow: float = 1.0   # alpha: rotations over L below which f_i / s is used
+
+
+def rope_freqs(rope_dim: int, theta) -> np.ndarray:
+    """Frequencies of the rope_dim / 2 rotary pairs: theta**(-2i/r), or their
+    YaRN interpolation when `theta` is a YaRN spec with factor > 1."""
+    i = np.arange(rope_dim // 2, dtype=np.float64)
+    if not isinstance(theta, YaRN):
+        return np.power(float(theta), -2.0 * i / rope_dim)
+    f = np.power(float(theta.theta), -2.0 * i / rope_dim)
+    if theta.factor <= 1.0:
+        return f
+    turns = theta.orig_ctx * f / (2.0 * math.pi)
+    gamma = np.clip((turns - theta.beta_slow) / (theta.beta_fast - theta.beta_slow), 0.0, 1.0)
+    return (1.0 - gamma) * f / theta.factor + gamma * f
+
+
+def attention_temperature(theta) -> float:
+    """Factor on the softmax logits: (0.1 ln s + 1)**2 under YaRN, else 1."""
+    if isinstance(theta, YaRN) and theta.factor > 1.0:
+        return (0.1 * math.log(theta.factor) + 1.0) ** 2
+    return 1.0
+
+
+# --------------------------------------------------------------------------
 # Partial RoPE ("Partial RoPE" row: last 64 of 512 dims; output rotated by -i)
 # --------------------------------------------------------------------------
-def rope(x: np.ndarray, pos, rope_dim: int, theta: float) -> np.ndarray:
+def rope(x: np.ndarray, pos, rope_dim: int, theta) -> np.ndarray:
     """Rotate the trailing `rope_dim` dims of x[..., d] at position(s) `pos`.
 
-    Pair i = dims (d - r + 2i, d - r + 2i + 1), angle pos * theta**(-2i/r);
+    Pair i = dims (d - r + 2i, d - r + 2i + 1), angle pos * f_i with
+    f_i = theta**(-2i/r) (or the YaRN frequencies, see rope_freqs);
     (a, b) -> (a cos - b sin, a sin + b cos).  `pos` broadcasts against
     x.shape[:-1].  A negative position gives the inverse rotation.
     """
@@ -99,8 +152,7 @@ def rope(x: np.ndarray, pos, rope_dim: int, theta: float) -> np.ndarray:
     if rope_dim == 0:
         return x
     d = x.shape[-1]
-    i = np.arange(rope_dim // 2, dtype=np.float64)
-    freq = np.power(float(theta), -2.0 * i / rope_dim)
+    freq = rope_freqs(rope_dim, theta)
     ang = np.asarray(pos, dtype=np.float64)[..., None] * freq
     c, s = np.cos(ang), np.sin(ang)
     a = x[..., d - rope_dim::2].copy()
@@ -115,7 +167,7 @@ def rope(x: np.ndarray, pos, rope_dim: int, theta: float) -> np.ndarray:
 # tokens at stride 4 with a per-channel softmax; HCA row: 128 tokens -> 1)
 # --------------------------------------------------------------------------
 def compress(x: np.ndarray, g: np.ndarray, width: int, stride: int,
-             rope_dim: int, theta: float, pos_offset: int = 0) -> np.ndarray:
+             rope_dim: int, theta, pos_offset: int = 0) -> np.ndarray:
     """Pool x[T, d] into N entries with per-channel softmax weights over the
     `width` taps of each entry, then rotate entry j at stride*j + pos_offset."""
     x = np.asarray(x, dtype=np.float64)
@@ -133,7 +185,7 @@ def compress(x: np.ndarray, g: np.ndarray, width: int, stride: int,
     return rope(out, pos, rope_dim, theta)
 
 
-def rotate_raw(x: np.ndarray, pos0: int, rope_dim: int, theta: float) -> np.ndarray:
+def rotate_raw(x: np.ndarray, pos0: int, rope_dim: int, theta) -> np.ndarray:
     """Raw (uncompressed) token rows rotated at their own positions."""
     x = np.asarray(x, dtype=np.float64)
     return rope(x, pos0 + np.arange(x.shape[0], dtype=np.int64), rope_dim, theta)
@@ -191,12 +243,14 @@ def index_topk(q_idx, w, k_idx, q_pos, n_cmp: int, width: int, stride: int,
 # sink in the denominator and the inverse output rotation
 # --------------------------------------------------------------------------
 def attend(q: np.ndarray, t: int, rows: np.ndarray, sink: np.ndarray, scale: float,
-           rope_dim: int, theta: float) -> np.ndarray:
+           rope_dim: int, theta) -> np.ndarray:
     """One query token.  q [H, d] (unrotated), rows [R, d] (rotated entries,
     each both key and value), sink [H].
 
     a_i = exp(z_i) / (exp(sink_h) + sum_i exp(z_i)), z_i = scale * (R(t) q_h) . r_i
-    o_h = sum_i a_i r_i, then the trailing rope dims of o_h rotated at -t."""
+    o_h = sum_i a_i r_i, then the trailing rope dims of o_h rotated at -t.
+    Under YaRN the scale carries the attention temperature."""
+    scale = scale * attention_temperature(theta)
     qh = rope(q, t, rope_dim, theta)
     sink = np.asarray(sink, dtype=np.float64)
     rows = np.asarray(rows, dtype=np.float64)

@@ -12,12 +12,39 @@ import cmath
 import math
 
 
+def _freq(i, rope_dim, theta):
+    """Frequency of rotary pair i.  `theta` is a base, or a tuple
+    (base, s, L, beta, alpha) for YaRN (Peng et al. 2023, section 3): the
+    pair turns L * w / (2 pi) times over L tokens; below alpha turns it runs
+    s times slower, above beta it is unchanged, linear blend in between."""
+    if not isinstance(theta, tuple):
+        return theta ** (-(2.0 * i) / rope_dim)
+    base, s, L, beta, alpha = theta
+    w = base ** (-(2.0 * i) / rope_dim)
+    if s <= 1.0:
+        return w
+    turns = L / (2.0 * math.pi / w)
+    if turns < alpha:
+        return w / s
+    if turns > beta:
+        return w
+    blend = (turns - alpha) / (beta - alpha)
+    return w / s * (1.0 - blend) + w * blend
+
+
+def temperature(theta):
+    """YaRN's factor on the logits, sqrt(1/t) = 0.1 ln s + 1; 1 otherwise."""
+    if isinstance(theta, tuple) and theta[1] > 1.0:
+        return (1.0 + 0.1 * math.log(theta[1])) ** 2
+    return 1.0
+
+
 def _rot(vec, pos, rope_dim, theta):
     d = len(vec)
     out = list(vec)
     base = d - rope_dim
     for i in range(rope_dim // 2):
-        w = theta ** (-(2.0 * i) / rope_dim)
+        w = _freq(i, rope_dim, theta)
         z = complex(vec[base + 2 * i], vec[base + 2 * i + 1]) * cmath.exp(1j * pos * w)
         out[base + 2 * i] = z.real
         out[base + 2 * i + 1] = z.imag
@@ -65,7 +92,8 @@ def attend(q, t, rows, sink, scale, rope_dim, theta):
     out = []
     for h, qv in enumerate(q):
         qr = _rot(qv, t, rope_dim, theta)
-        z = [scale * sum(a * b for a, b in zip(qr, r)) for r in rows]
+        tau = temperature(theta)
+        z = [tau * scale * sum(a * b for a, b in zip(qr, r)) for r in rows]
         mx = max(z + [sink[h]])
         ex = [math.exp(v - mx) for v in z]
         den = math.exp(sink[h] - mx) + sum(ex)

@@ -323,3 +323,91 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(oracle, "attend", no_sink)
     with pytest.raises(AssertionError):
         test_sink_closed_form_and_weight_sum()
+
+
+# ---------------------------------------------------------------- YaRN
+# The compressed layers' extended RoPE ("Partial RoPE" rows: theta = 160,000
+# with YaRN, factor 16 over 65,536 tokens), pinned to what the published
+# definition fixes (Peng et al. 2023, section 3) without retyping it: the
+# end points of the ramp, its bounds, the temperature's closed form, the
+# rotation's relative-distance property and the pure-Python brute force.
+V4_YARN = oracle.YaRN(theta=160000.0, factor=16.0, orig_ctx=65536)
+V4_YARN_TUPLE = (160000.0, 16.0, 65536, 32.0, 1.0)
+
+
+def test_yarn_with_factor_one_is_plain_rope():
+    x = _rng(40).standard_normal((5, 32))
+    pos = np.array([0, 3, 70000, 1 << 20, -9])
+    plain = oracle.rope(x, pos, 16, 160000.0)
+    spec = oracle.YaRN(theta=160000.0, factor=1.0, orig_ctx=65536)
+    np.testing.assert_array_equal(oracle.rope(x, pos, 16, spec), plain)
+    assert oracle.attention_temperature(spec) == 1.0
+
+
+def test_yarn_keeps_the_fastest_pair_and_slows_the_slowest_by_the_factor():
+    f = oracle.rope_freqs(64, V4_YARN)
+    base = 160000.0 ** (-np.arange(32) * 2.0 / 64)
+    # pair 0 turns once per token: 65,536 / (2 pi) >> 32 turns over the context
+    assert f[0] == 1.0
+    # pair 31 turns 0.1 times over 65,536 tokens (< 1): interpolated by 16
+    assert 65536 * base[31] / (2 * math.pi) < 1.0
+    assert f[31] == base[31] / 16.0
+    # every pair lies between its interpolated and original frequency, and
+    # the interpolation never speeds a pair up
+    assert np.all(f <= base * (1 + 1e-15)) and np.all(f >= base / 16.0 * (1 - 1e-15))
+    assert np.all(np.diff(f / base) <= 1e-15)  # slower pairs are interpolated more
+
+
+def test_yarn_temperature_closed_form_and_one_key_attention():
+    tau = oracle.attention_temperature(V4_YARN)
+    assert tau == pytest.approx((1 + 0.1 * math.log(16.0)) ** 2, rel=1e-15)
+    assert tau == pytest.approx(1.63139, abs=1e-5)
+    # one key e at position p, no rope dims rotated for the dot product
+    # check: with rope_dim 0, a = exp(tau s z) / (exp(sink) + exp(tau s z))
+    rng = _rng(41)
+    q, e, sink = rng.standard_normal((3, 8)), rng.standard_normal((1, 8)), rng.standard_normal(3)
+    out = oracle.attend(q, 50, e, sink, 0.25, 0, V4_YARN)
+    z = tau * 0.25 * (q @ e[0])
+    a = np.exp(z) / (np.exp(sink) + np.exp(z))
+    np.testing.assert_allclose(out, a[:, None] * e, rtol=0, atol=1e-14)
+
+
+def test_yarn_rotation_depends_only_on_relative_distance():
+    rng = _rng(42)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for a, b, shift in ((10, 3, 1000), (70000, 5, 123456), (0, 300000, 77)):
+        d0 = oracle.rope(q, a, 64, V4_YARN) @ oracle.rope(k, b, 64, V4_YARN)
+        d1 = oracle.rope(q, a + shift, 64, V4_YARN) @ oracle.rope(k, b + shift, 64, V4_YARN)
+        assert d0 == pytest.approx(d1, rel=1e-9, abs=1e-9)
+    back = oracle.rope(oracle.rope(q, 98765, 64, V4_YARN), -98765, 64, V4_YARN)
+    np.testing.assert_allclose(back, q, atol=1e-12)
+
+
+def test_yarn_layer_matches_brute_force():
+    # a tiny layer whose positions run past the original context (L = 40)
+    L = _tiny_layer(43, T=96)
+    kw = dict(L["kw"])
+    # rope_dim 8, base 500, L 40: pair 0 turns 6.4 times over L (kept, above
+    # beta = 4), pair 1 1.3 times (on the ramp), pairs 2-3 under once (slowed)
+    spec = oracle.YaRN(theta=500.0, factor=4.0, orig_ctx=40, beta_fast=4.0, beta_slow=1.0)
+    tup = (500.0, 4.0, 40, 4.0, 1.0)
+    kw["theta"] = spec
+    kv_cmp, kv_raw, idx, out = oracle.csa_prefill_layer(
+        L["x"], L["g"], L["q_idx"], L["w"], L["k_idx"], L["q"], L["sink"], **kw)
+    b_cmp = brute.compress(L["x"].tolist(), L["g"].tolist(), kw["width"], kw["stride"],
+                           kw["rope_dim"], tup)
+    np.testing.assert_allclose(kv_cmp, np.array(b_cmp), atol=1e-12)
+    T = L["x"].shape[0]
+    for t in (0, 7, 40, 95):
+        sel = [j for j in idx[t].tolist() if j >= 0]
+        raw = [brute._rot(list(L["x"][u]), u, kw["rope_dim"], tup)
+               for u in brute.window(t, kw["window"], 0, T)]
+        rows = [b_cmp[j] for j in sel] + raw
+        ref = brute.attend(L["q"][t].tolist(), t, rows, L["sink"].tolist(), kw["scale"],
+                           kw["rope_dim"], tup)
+        np.testing.assert_allclose(out[t], np.array(ref), atol=1e-12)
+    # the ramp of this spec is exercised: some pairs interpolated, some kept
+    f = oracle.rope_freqs(kw["rope_dim"], spec)
+    plain = oracle.rope_freqs(kw["rope_dim"], 500.0)
+    assert f[0] == plain[0] and plain[1] / 4 < f[1] < plain[1]
+    np.testing.assert_array_equal(f[2:], plain[2:] / 4)
