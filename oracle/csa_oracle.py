@@ -46,7 +46,12 @@ Readings of points the pages leave open:
 * top-k keeps the k largest scores, ties to the lower index, returned in
   ascending index order and padded with -1; with fewer than k visible
   entries all are kept;
-* no de-duplication between window rows and compressed entries.
+* no de-duplication between window rows and compressed entries;
+* CSA2 ("DeepSeek-V4.1-Flash vs Inkling", row "CSA2 encoder layers (2x
+  compression, Full + Reuse)": KV pooled 2 -> 1, computed in 3 of 18 layers,
+  the rest reuse that KV and its top-512 selection): a Full layer is this
+  layer with width = stride = 2 and k = 512; a Reuse layer is sparse_attn
+  with its own queries (and sink) over the Full layer's entries and indices.
 
 Parity unpinned by the pages (conventions fixed here and given to the GPU
 path as parameters): entry position, RoPE pair layout, window inclusivity,

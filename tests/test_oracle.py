@@ -28,7 +28,7 @@ def _rng(seed):
 def test_entry_counts_match_stated_workloads():
     rows = [l.split() for l in open(os.path.join(GOLDEN, "entry_counts.txt"))
             if l.strip() and not l.startswith("#")]
-    assert len(rows) == 5
+    assert len(rows) == 6
     for T, w, s, n in (map(int, r) for r in rows):
         assert oracle.n_compressed(T, w, s) == n
 
@@ -411,3 +411,33 @@ def test_yarn_layer_matches_brute_force():
     plain = oracle.rope_freqs(kw["rope_dim"], 500.0)
     assert f[0] == plain[0] and plain[1] / 4 < f[1] < plain[1]
     np.testing.assert_array_equal(f[2:], plain[2:] / 4)
+
+
+# ---------------------------------------------------------------- CSA2
+def test_csa2_full_and_reuse_layers_match_brute_force():
+    # "CSA2 encoder layers (2x compression, Full + Reuse)": KV pooled 2 -> 1
+    # and computed in a Full layer; a Reuse layer attends with its own
+    # queries over the Full layer's entries and top-k selection
+    L = _tiny_layer(44, T=40, width=2, stride=2, k=6)
+    kw = L["kw"]
+    T = L["x"].shape[0]
+    kv_cmp, kv_raw, idx, out = oracle.csa_prefill_layer(
+        L["x"], L["g"], L["q_idx"], L["w"],
+        _rng(45).integers(-3, 4, size=(T // 2, L["q_idx"].shape[2])).astype(np.float64),
+        L["q"], L["sink"], **kw)
+    assert kv_cmp.shape[0] == T // 2  # non-overlapping pairs: floor(T / 2) entries
+    b_cmp = brute.compress(L["x"].tolist(), L["g"].tolist(), 2, 2, kw["rope_dim"], THETA)
+    np.testing.assert_allclose(kv_cmp, np.array(b_cmp), atol=1e-12)
+    q2 = _rng(46).standard_normal(L["q"].shape)
+    sink2 = _rng(47).standard_normal(L["sink"].shape)
+    reuse = oracle.sparse_attn(q2, np.arange(T), kv_cmp, idx, kv_raw, 0, T, sink2, kw["scale"],
+                               kw["window"], kw["rope_dim"], THETA)
+    for t in (0, 1, 2, 17, 39):
+        sel = [j for j in idx[t].tolist() if j >= 0]
+        assert all(2 * j + 1 <= t for j in sel)  # a pair is visible once both tokens are
+        raw = [brute._rot(list(L["x"][u]), u, kw["rope_dim"], THETA)
+               for u in brute.window(t, kw["window"], 0, T)]
+        rows = [b_cmp[j] for j in sel] + raw
+        ref = brute.attend(q2[t].tolist(), t, rows, sink2.tolist(), kw["scale"], kw["rope_dim"],
+                           THETA)
+        np.testing.assert_allclose(reuse[t], np.array(ref), atol=1e-12)
