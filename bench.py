@@ -79,7 +79,9 @@ def _args():
     ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
     ap.add_argument("--workload", default=HEADLINE,
                     help="csa_decode_bs32_ctx65536 (default), csa_decode_bs4_ctx1048576, "
-                         "hca_decode_bs16_ctx131072 or csa_prefill_T8192")
+                         "hca_decode_bs16_ctx131072, csa_prefill_T8192, "
+                         "csa_decode_yarn_bs32_ctx131072 or csa2_decode_bs32_ctx65536 "
+                         "(one Full + five Reuse layers)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--seq-len", type=int, default=0,
@@ -121,6 +123,12 @@ def _config(wl, extra=None, flush_mib=256):
          "parallelism": "replicas"}
     if wl.kind != "hca_decode":
         c.update({"indexer": f"{wl.idx_heads}x{wl.idx_dim}", "topk": wl.topk})
+    if wl.rope_factor > 1.0:
+        c["rope"] = (f"theta {wl.theta:g}, YaRN factor {wl.rope_factor:g} over "
+                     f"{wl.rope_orig_ctx} tokens")
+    if wl.reuse_layers:
+        c["layers"] = (f"1 Full layer (indexer, top-k, attention) + {wl.reuse_layers} Reuse "
+                       "layers (attention over the Full layer's entries and selection)")
     if extra:
         c.update(extra)
     return c
@@ -163,7 +171,10 @@ def algorithmic_work(wl):
     g["topk_select"] = {"bytes": scores + sel, "flops": 0}
     g["sparse_attn"] = {"bytes": rows + q + out + sel + H * 4,
                         "flops": int(4 * n_q * H * n_rows * d)}
-    # the step's own bytes: scores and indices stay between its kernels
+    if wl.reuse_layers:
+        g["reuse_attn"] = {k: wl.reuse_layers * v for k, v in g["sparse_attn"].items()}
+    # the step's own bytes: scores and indices stay between its kernels (each
+    # Reuse layer reads the selection again)
     g["step"] = {"bytes": sum(v["bytes"] for v in g.values()) - 2 * scores - 2 * sel}
     return g
 
@@ -253,19 +264,22 @@ def _oracle_sample(wl):
     from sparse_compressed_attention_csa_b200 import workloads as W
     f = W.to_f64
     v = W.bits_to_f32
+    th = wl.theta if wl.rope_factor <= 1.0 else oracle.YaRN(
+        theta=wl.theta, factor=wl.rope_factor, orig_ctx=wl.rope_orig_ctx,
+        beta_fast=wl.rope_beta_fast, beta_slow=wl.rope_beta_slow)
     if wl.kind == "csa_prefill":
         data = W.generate(wl)
         rows = np.linspace(0, wl.T - 1, 16).astype(np.int64)
 
         def step():
             kv = oracle.compress(f(data["x"][0]), f(data["g"][0]), wl.width, wl.stride,
-                                 wl.rope_dim, wl.theta, wl.pos_offset)
-            raw = oracle.rotate_raw(f(data["x"][0]), 0, wl.rope_dim, wl.theta)
+                                 wl.rope_dim, th, wl.pos_offset)
+            raw = oracle.rotate_raw(f(data["x"][0]), 0, wl.rope_dim, th)
             qp = data["q_pos"][0]
             idx = oracle.index_topk(v(data["q_idx"][0]), data["w"][0], f(data["k_idx"][0]), qp,
                                     kv.shape[0], wl.width, wl.stride, wl.topk, rows)
             return oracle.sparse_attn(f(data["q"][0][rows]), qp[rows], kv, idx, raw, 0, wl.T,
-                                      data["sink"], wl.scale, wl.window, wl.rope_dim, wl.theta)
+                                      data["sink"], wl.scale, wl.window, wl.rope_dim, th)
         return step, len(rows) * wl.n_heads, (
             "compression of the whole sequence, then the indexer, top-k and 128-head attention "
             "for 16 of the 8,192 query tokens, fp64 NumPy oracle")
@@ -276,22 +290,28 @@ def _oracle_sample(wl):
             return oracle.hca_attn(f(data["q"][0]), data["q_pos"][0], v(data["kv_cmp"][0]),
                                    int(data["n_cmp"][0]), v(data["kv_raw"][0]),
                                    int(data["raw_pos0"][0]), int(data["n_raw"][0]), data["sink"],
-                                   wl.scale, wl.window, wl.width, wl.stride, wl.rope_dim,
-                                   wl.theta)
+                                   wl.scale, wl.window, wl.width, wl.stride, wl.rope_dim, th)
         return step, wl.n_heads, (f"one of the {wl.B} sequences per step (128-head attention "
                                   f"over its {wl.n_cmp} entries and window), fp64 NumPy oracle")
+
+    def attend(q, idx, sink):
+        return oracle.sparse_attn(q, data["q_pos"][0], v(data["kv_cmp"][0]), idx,
+                                  v(data["kv_raw"][0]), int(data["raw_pos0"][0]),
+                                  int(data["n_raw"][0]), sink, wl.scale, wl.window,
+                                  wl.rope_dim, th)
 
     def step():
         qp = data["q_pos"][0]
         idx = oracle.index_topk(f(data["q_idx"][0]), data["w"][0], f(data["k_idx"][0]), qp,
                                 int(data["n_cmp"][0]), wl.width, wl.stride, wl.topk)
-        return oracle.sparse_attn(f(data["q"][0]), qp, v(data["kv_cmp"][0]), idx,
-                                  v(data["kv_raw"][0]), int(data["raw_pos0"][0]),
-                                  int(data["n_raw"][0]), data["sink"], wl.scale, wl.window,
-                                  wl.rope_dim, wl.theta)
-    return step, wl.n_heads, (f"one of the {wl.B} sequences per step (indexer over "
-                              f"{wl.n_cmp:,} entries, top-{wl.topk}, 128-head attention), "
-                              f"fp64 NumPy oracle")
+        outs = [attend(f(data["q"][0]), idx, data["sink"])]
+        for r in range(wl.reuse_layers):
+            outs.append(attend(f(data["q_reuse"][r][0]), idx, data["sink_reuse"][r]))
+        return outs
+    reuse = f" + {wl.reuse_layers} Reuse layers" if wl.reuse_layers else ""
+    return step, wl.n_heads * (1 + wl.reuse_layers), (
+        f"one of the {wl.B} sequences per step (indexer over {wl.n_cmp:,} entries, "
+        f"top-{wl.topk}, 128-head attention{reuse}), fp64 NumPy oracle")
 
 
 def run_reference(args, rank):
@@ -385,7 +405,9 @@ def run_cuda(args, rank, world, local):
     t = {k: todev(v) for k, v in data.items()}
     p = L.Params(d=wl.d, rope_dim=wl.rope_dim, theta=wl.theta, scale=wl.scale,
                  n_heads=wl.n_heads, idx_heads=wl.idx_heads, idx_dim=wl.idx_dim, topk=wl.topk,
-                 window=wl.window, width=wl.width, stride=wl.stride, pos_offset=wl.pos_offset)
+                 window=wl.window, width=wl.width, stride=wl.stride, pos_offset=wl.pos_offset,
+                 rope_factor=wl.rope_factor, rope_orig_ctx=wl.rope_orig_ctx,
+                 rope_beta_fast=wl.rope_beta_fast, rope_beta_slow=wl.rope_beta_slow)
     Bsz, Tq, N = wl.B, wl.Tq, wl.n_cmp
     out = torch.empty_like(t["q"])
     ops = {"hca_decode": [L.CSA_OP_HCA_ATTN]}.get(
@@ -416,6 +438,15 @@ def run_cuda(args, rank, world, local):
         groups.append(("sparse_attn", lambda: L.csa_sparse_attn(
             p, t["q"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"], t["n_raw"],
             t["sink"], out, ws)))
+    R = wl.reuse_layers
+    if R:
+        out_r = torch.empty_like(t["q_reuse"])
+
+        def reuse_layers():
+            for r in range(R):
+                L.csa_sparse_attn(p, t["q_reuse"][r], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"],
+                                  t["raw_pos0"], t["n_raw"], t["sink_reuse"][r], out_r[r], ws)
+        groups.append(("reuse_attn", reuse_layers))
 
     mib = max(args.flush_mib, 0)
     flush = torch.empty(mib << 20, dtype=torch.uint8, device=dev)
@@ -495,22 +526,23 @@ def run_cuda(args, rank, world, local):
     n_bd = min(args.steps, 200)
     bd = breakdown(n_bd)
     step_ms_max = max_over_ranks(step_ms, world, dev)
-    qh_per_step = wl.B * wl.Tq * wl.n_heads
+    qh_per_step = wl.B * wl.Tq * wl.n_heads * (1 + R)
     value = job_throughput(qh_per_step, world, step_ms_max)
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host
     h2d_keys = {"csa_decode": ("q", "q_idx", "w", "q_pos"), "hca_decode": ("q", "q_pos"),
-                "csa_prefill": ("x", "g", "q_idx", "w", "q")}[wl.kind]
+                "csa_prefill": ("x", "g", "q_idx", "w", "q")}[wl.kind] + (("q_reuse",) if R else ())
     h_in = {k: torch.from_numpy(np.ascontiguousarray(data[k].view(np.int16) if data[k].dtype ==
                                                       np.uint16 else data[k])).pin_memory()
             for k in h2d_keys}
     d_in = {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=dev) for k in h_in}
     h_out = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+    h_out_r = torch.empty(out_r.shape, dtype=torch.int16).pin_memory() if R else None
     lw = layer.Workspace(dev)
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     h2d = sum(h_in[k].numel() * h_in[k].element_size() for k in h_in)
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = h_out.numel() * h_out.element_size() + (h_out_r.numel() * 2 if R else 0)
 
     def bf(k):
         return d_in[k].view(torch.bfloat16)
@@ -526,6 +558,12 @@ def run_cuda(args, rank, world, local):
                                         t["k_idx"], t["n_cmp"], t["kv_cmp"], t["kv_raw"],
                                         t["raw_pos0"], t["n_raw"], t["sink"], lw, idx=idx,
                                         out=out)
+                for r in range(R):
+                    layer.reuse_attn(p, bf("q_reuse")[r], d_in["q_pos"], t["kv_cmp"], idx,
+                                     t["kv_raw"], t["raw_pos0"], t["n_raw"], t["sink_reuse"][r],
+                                     lw, out=out_r[r])
+                if R:
+                    h_out_r.copy_(out_r.view(torch.int16), non_blocking=True)
             elif wl.kind == "hca_decode":
                 o = layer.hca_decode(p, bf("q"), d_in["q_pos"], t["kv_cmp"], t["n_cmp"],
                                      t["kv_raw"], t["raw_pos0"], t["n_raw"], t["sink"], lw,

@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define CSA_ABI_VERSION 1
+#define CSA_ABI_VERSION 2
 
 typedef enum {
   CSA_OK = 0,
@@ -92,7 +92,19 @@ typedef enum {
 /* Layer constants.  Defaults of the measured model: d 512, rope_dim 64,
  * theta 1e4, scale 1/sqrt(512), n_heads 128, idx_heads 64, idx_dim 128,
  * topk 1024, window 128, (width, stride) = (8, 4) for CSA and (128, 128)
- * for HCA, pos_offset 0. */
+ * for HCA, pos_offset 0, rope_factor 1 (plain RoPE).
+ *
+ * Extended RoPE ("DeepSeek-V4-Pro vs Inkling", "Partial RoPE" row: the
+ * compressed layers use theta = 160,000 with YaRN, factor 16 over 65,536
+ * tokens).  With rope_factor s > 1 every rotation of the call (queries,
+ * entries, window rows, the output's inverse rotation) uses the YaRN
+ * frequencies of Peng et al. 2023 ("YaRN: Efficient Context Window
+ * Extension of Large Language Models", section 3): rotary pair i with
+ * f_i = theta^(-2i/rope_dim) turns n_i = rope_orig_ctx * f_i / (2 pi) times
+ * over the original context; with g = clamp((n_i - rope_beta_slow) /
+ * (rope_beta_fast - rope_beta_slow), 0, 1) it rotates at (1 - g) f_i / s +
+ * g f_i.  The attention calls then multiply `scale` by YaRN's temperature
+ * (0.1 ln s + 1)^2.  The paper's beta values are 32 (fast) and 1 (slow). */
 typedef struct {
   int32_t d;          /* entry / head dim, multiple of 32, <= 1024 */
   int32_t rope_dim;   /* rotated trailing dims, even, <= d (0 = no RoPE) */
@@ -106,6 +118,10 @@ typedef struct {
   int32_t width;      /* pooling width w_c */
   int32_t stride;     /* pooling stride m */
   int32_t pos_offset; /* RoPE position of entry j is stride*j + pos_offset */
+  float rope_factor;    /* YaRN factor s (<= 1: plain RoPE, the fields below unused) */
+  int32_t rope_orig_ctx;  /* YaRN original context length L (>= 1 when s > 1) */
+  float rope_beta_fast; /* YaRN beta: pairs turning more often over L keep f_i */
+  float rope_beta_slow; /* YaRN alpha: pairs turning less often over L get f_i / s */
 } csa_params_t;
 
 /* Library ABI version (CSA_ABI_VERSION). */
@@ -244,6 +260,12 @@ uint64_t csa_launch_count(void);
 /* Synchronizes `stream`, then reads and clears the current device's error
  * word: CSA_OK, CSA_ERR_DEVICE_TIMEOUT or CSA_ERR_DEVICE_BOUNDS. */
 csa_status_t csa_poll_device_error(void* stream);
+
+/* The source line, in the library's kernel sources, of the device-side check
+ * that recorded the error the last failing csa_poll_device_error() returned
+ * (in this process, on any device); 0 before any.  A diagnostic: for a
+ * timeout it names the wait that ran out first. */
+int32_t csa_last_device_error_site(void);
 
 #ifdef __cplusplus
 }

@@ -38,7 +38,9 @@ class csa_params_t(ctypes.Structure):
                 ("scale", ctypes.c_float), ("n_heads", ctypes.c_int32),
                 ("idx_heads", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
                 ("topk", ctypes.c_int32), ("window", ctypes.c_int32), ("width", ctypes.c_int32),
-                ("stride", ctypes.c_int32), ("pos_offset", ctypes.c_int32)]
+                ("stride", ctypes.c_int32), ("pos_offset", ctypes.c_int32),
+                ("rope_factor", ctypes.c_float), ("rope_orig_ctx", ctypes.c_int32),
+                ("rope_beta_fast", ctypes.c_float), ("rope_beta_slow", ctypes.c_float)]
 
 
 @dataclass(frozen=True)
@@ -56,12 +58,17 @@ class Params:
     width: int = 8
     stride: int = 4
     pos_offset: int = 0
+    rope_factor: float = 1.0      # YaRN factor s (1: plain RoPE)
+    rope_orig_ctx: int = 0        # YaRN original context L
+    rope_beta_fast: float = 32.0  # YaRN beta
+    rope_beta_slow: float = 1.0   # YaRN alpha
 
     def c(self) -> csa_params_t:
         sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
         return csa_params_t(self.d, self.rope_dim, self.theta, sc, self.n_heads, self.idx_heads,
                             self.idx_dim, self.topk, self.window, self.width, self.stride,
-                            self.pos_offset)
+                            self.pos_offset, self.rope_factor, self.rope_orig_ctx,
+                            self.rope_beta_fast, self.rope_beta_slow)
 
 
 _lib = None
@@ -100,6 +107,8 @@ def _load():
     lib.csa_launch_count.argtypes = []
     lib.csa_set_wait_limit_ns.restype = None
     lib.csa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.csa_last_device_error_site.restype = ctypes.c_int32
+    lib.csa_last_device_error_site.argtypes = []
     for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
               "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error",
               "csa_index_topk_noalloc"):
@@ -282,3 +291,8 @@ def csa_set_wait_limit_ns(ns: int = 0):
 
 def csa_poll_device_error(stream=None):
     _check(_load().csa_poll_device_error(_stream(stream)))
+
+
+def csa_last_device_error_site() -> int:
+    """Kernel source line of the check behind the last device error polled."""
+    return int(_load().csa_last_device_error_site())

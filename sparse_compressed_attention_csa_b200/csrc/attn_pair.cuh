@@ -511,32 +511,37 @@ __global__ void __launch_bounds__(kApThreads, 1)
       for (int e = 8; e < 64; ++e) mx[e & 7] = fmaxf(mx[e & 7], z[e]);
       const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      if (mt > m_run + kApRescaleLog2 || m_run == -INFINITY) {
-        if (i > 0 && m_run != -INFINITY) {
-          // O holds P V of earlier tiles: wait for the last PV, then rescale
-          ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(i - 1) & 1],
-                                                 (uint32_t)((i - 1) >> 1) & 1u, abortp, wait_ns));
-          if (!ok) break;
-          tc_fence_after();
-          const float alpha = exp2f(m_run - mt);
+      // lazy rescale: a head's running maximum moves only when the tile's
+      // exceeds it by more than 2^8 (or on its first finite tile).  The
+      // decision is per head (lane), but the wait and the TMEM accesses are
+      // warp-collective: when any lane of the warp moves, the whole warp
+      // takes the branch, the lanes that keep their maximum with alpha = 1.
+      const bool move = mt > m_run + kApRescaleLog2 || m_run == -INFINITY;
+      const float m_new = move ? mt : m_run;
+      if (i > 0 && __any_sync(0xffffffffu, move && m_run != -INFINITY)) {
+        // O holds P V of earlier tiles: wait for the last PV, then rescale
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done[(i - 1) & 1],
+                                               (uint32_t)((i - 1) >> 1) & 1u, abortp, wait_ns));
+        if (!ok) break;
+        tc_fence_after();
+        const float alpha = (move && m_run != -INFINITY) ? exp2f(m_run - m_new) : 1.f;
 #pragma unroll 1
-          for (int cc = 0; cc < kApHalf; cc += 32) {
-            uint32_t r[32];
-            tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
-            tmem_wait_ld();
-            uint32_t w16[16];
+        for (int cc = 0; cc < kApHalf; cc += 32) {
+          uint32_t r[32];
+          tmem_ld32(t_o + lane_base + (uint32_t)cc, r);
+          tmem_wait_ld();
+          uint32_t w16[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st16(t_o + lane_base + (uint32_t)cc, w16);
+          for (int e = 0; e < 16; ++e) w16[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(t_o + lane_base + (uint32_t)cc, w16);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              w16[e] = __float_as_uint(__uint_as_float(r[16 + e]) * alpha);
-            tmem_st16(t_o + lane_base + (uint32_t)cc + 16, w16);
-          }
-          l_run *= alpha;
+          for (int e = 0; e < 16; ++e)
+            w16[e] = __float_as_uint(__uint_as_float(r[16 + e]) * alpha);
+          tmem_st16(t_o + lane_base + (uint32_t)cc + 16, w16);
         }
-        m_run = mt;
+        l_run *= alpha;
       }
+      m_run = m_new;
       uint32_t pk[32];
       float ps8[8];
 #pragma unroll
@@ -757,7 +762,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
               }
               if (mbar_try_wait(&sm.full[slot], fph)) break;
               if ((it & 63u) == 0u) {
-                if (*abortp) {
+                if (*abortp || timeout_recorded()) {
+                  *abortp = 1;
                   okm = false;
                   break;
                 }
@@ -791,8 +797,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
     // TMEM is freed only after every MMA issued here has landed: one commit
     // tracks them all
     tc_commit(&sm.mma_drain);
-    int never = 0;
-    mbar_wait(&sm.mma_drain, 0, &never, kApDrainNs);
+    mbar_drain(&sm.mma_drain, 0, kApDrainNs);
   }
 
   // ======================= wind-down
@@ -802,20 +807,17 @@ __global__ void __launch_bounds__(kApThreads, 1)
   __syncwarp();
   cluster_sync_all();
   if (threadIdx.x == 0) {
-    int never = 0;
     for (int i = x_recv; i < x_posted; ++i)
-      mbar_wait_cluster(&sm.xfull[i % kApXBufs], (uint32_t)(i / kApXBufs) & 1u, &never,
-                        kApDrainNs);
+      mbar_drain_cluster(&sm.xfull[i % kApXBufs], (uint32_t)(i / kApXBufs) & 1u, kApDrainNs);
   }
   if (warp == 4 && lane == 0) {
     // every copy into shared memory lands before the CTA may exit: q, and in
     // each ring slot the last chunk requested into it (an earlier one was
     // consumed before the slot could be refilled)
-    int never = 0;
-    mbar_wait(&sm.q_tma, 0, &never, kApDrainNs);
+    mbar_drain(&sm.q_tma, 0, kApDrainNs);
     for (int s = 0; s < kApSlots; ++s) {
       const int n = sm.last_n[s];
-      if (n >= 0) mbar_wait(&sm.full[s], (uint32_t)(n / kApSlots) & 1u, &never, kApDrainNs);
+      if (n >= 0) mbar_drain(&sm.full[s], (uint32_t)(n / kApSlots) & 1u, kApDrainNs);
     }
   }
   tc_fence_before();

@@ -29,18 +29,18 @@ struct AttnArgs {
   int raw_max;
   const float* sink;
   int B, Tq, H, d, rope_dim, topk, window, width, stride;
-  float scale;
-  double theta;
+  float scale;  // with the extended RoPE's temperature
+  RopeSpec rope;
   void* out;
 };
 
 // Rotate the lane's values (dims c = lane + 32*k) at position pos: pairs
 // (2i, 2i+1) of the rope range sit in neighbouring lanes.
 template <int NK>
-__device__ __forceinline__ void rotate_lane_dims(float* v, int d, int rope_dim, long long pos,
-                                                 double theta) {
+__device__ __forceinline__ void rotate_lane_dims(float* v, int d, const RopeSpec& rope,
+                                                 long long pos) {
   const int lane = threadIdx.x & 31;
-  const int rope0 = d - rope_dim;
+  const int rope0 = d - rope.rope_dim;
 #pragma unroll
   for (int k = 0; k < NK; ++k) {
     const int c = lane + 32 * k;
@@ -48,7 +48,7 @@ __device__ __forceinline__ void rotate_lane_dims(float* v, int d, int rope_dim, 
     const float other = __shfl_xor_sync(0xffffffffu, v[k], 1);
     if (active) {
       float cs, sn;
-      rope_cos_sin(pos, (c - rope0) >> 1, rope_dim, theta, &cs, &sn);
+      rope_cos_sin(pos, rope_freq(rope, (c - rope0) >> 1), &cs, &sn);
       v[k] = (c & 1) ? (other * sn + v[k] * cs) : (v[k] * cs - other * sn);
     }
   }
@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(32 * kAttnSimtWarps) k_attn_simt(AttnArgs a) {
   float qv[NK];
   const T* qp = reinterpret_cast<const T*>(a.q) + ((size_t)row * a.H + h) * d;
   _Pragma("unroll") for (int k = 0; k < NK; ++k) qv[k] = to_f32(qp[lane + 32 * k]);
-  rotate_lane_dims<NK>(qv, d, a.rope_dim, t, a.theta);
+  rotate_lane_dims<NK>(qv, d, a.rope, t);
 
   // rows: n_sel compressed entries, then the window's raw rows
   int n_sel;
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(32 * kAttnSimtWarps) k_attn_simt(AttnArgs a) {
     for (int w = 0; w < kAttnSimtWarps; ++w) s = fmaf(sm_acc[w][lane + 32 * k], scl[w], s);
     o[k] = s * inv;
   }
-  rotate_lane_dims<NK>(o, d, a.rope_dim, -(long long)t, a.theta);
+  rotate_lane_dims<NK>(o, d, a.rope, -(long long)t);
   T* op = reinterpret_cast<T*>(a.out) + ((size_t)row * a.H + h) * d;
   _Pragma("unroll") for (int k = 0; k < NK; ++k) store(op + lane + 32 * k, o[k]);
 }

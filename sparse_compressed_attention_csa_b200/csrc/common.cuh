@@ -10,11 +10,15 @@
 namespace csa {
 
 // Per-device error word: kernels record the first device-side failure here
-// (a bounded wait that ran out, a failed index check); csa_poll_device_error
-// reads and clears it.  Never trap: the context stays usable.
+// (a bounded wait that ran out, a failed index check), and beside it the
+// source line of the check that recorded it; csa_poll_device_error reads and
+// clears both.  Never trap: the context stays usable.
 __device__ int g_device_error;
+__device__ int g_device_error_site;
 
-__device__ __forceinline__ void report_error(int code) { atomicCAS(&g_device_error, 0, code); }
+__device__ __forceinline__ void report_error(int code, int site = __builtin_LINE()) {
+  if (atomicCAS(&g_device_error, 0, code) == 0) atomicExch(&g_device_error_site, site);
+}
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -33,14 +37,37 @@ __device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 
-// RoPE ("Partial RoPE" row: rotate the trailing rope_dim of d dims).  Pair i
-// is dims (d - rope_dim + 2i, d - rope_dim + 2i + 1), frequency
-// theta^(-2i/rope_dim), angle pos * frequency.  The angle and its sine and
-// cosine are taken in double precision so that positions up to 2^20 keep
-// full fp32 accuracy in the rotation.
-__device__ __forceinline__ void rope_cos_sin(long long pos, int i, int rope_dim, double theta,
-                                             float* c, float* s) {
-  double freq = pow(theta, -2.0 * (double)i / (double)rope_dim);
+// RoPE ("Partial RoPE" row: rotate the trailing rope_dim of d dims).  Pair
+// i is dims (d - rope_dim + 2i, d - rope_dim + 2i + 1), angle pos * f_i.
+// f_i = theta^(-2i/rope_dim), or, for the compressed layers' extended RoPE
+// (same row: theta 160,000 with YaRN, factor 16 over 65,536 tokens), the
+// YaRN frequency of the published definition (Peng et al. 2023, section 3):
+// a pair that turns n_i = L f_i / (2 pi) times over the original context L
+// gets (1 - g) f_i / s + g f_i with g = clamp((n_i - alpha) / (beta - alpha),
+// 0, 1).
+struct RopeSpec {
+  int rope_dim;
+  double theta;
+  double factor;    // s; <= 1: plain RoPE
+  double orig_ctx;  // L
+  double beta_fast; // beta
+  double beta_slow; // alpha
+};
+
+__host__ __device__ inline double rope_freq(const RopeSpec& r, int i) {
+  double f = pow(r.theta, -2.0 * (double)i / (double)r.rope_dim);
+  if (r.factor > 1.0) {
+    const double turns = r.orig_ctx * f / 6.283185307179586;
+    double g = (turns - r.beta_slow) / (r.beta_fast - r.beta_slow);
+    g = g < 0.0 ? 0.0 : (g > 1.0 ? 1.0 : g);
+    f = (1.0 - g) * f / r.factor + g * f;
+  }
+  return f;
+}
+
+// cos / sin of pos * freq, the angle and its sine and cosine taken in double
+// precision so that positions up to 2^20 keep full fp32 accuracy.
+__device__ __forceinline__ void rope_cos_sin(long long pos, double freq, float* c, float* s) {
   double sd, cd;
   sincos((double)pos * freq, &sd, &cd);
   *c = (float)cd;

@@ -16,13 +16,13 @@ namespace csa {
 template <typename T>
 __global__ void __launch_bounds__(256) k_compress(const T* __restrict__ x, const T* __restrict__ g,
                                                   int T_len, int d, int N, int width, int stride,
-                                                  int rope_dim, double theta, int pos_offset,
+                                                  RopeSpec rope, int pos_offset,
                                                   T* __restrict__ kv_cmp, T* __restrict__ kv_raw) {
   const int b = blockIdx.y;
   const int r = blockIdx.x;
   const T* xb = x + (size_t)b * T_len * d;
   const T* gb = g + (size_t)b * T_len * d;
-  const int rope0 = d - rope_dim;
+  const int rope0 = d - rope.rope_dim;
   if (r < N) {
     const long long pos = (long long)stride * r + pos_offset;
     T* dst = kv_cmp + ((size_t)b * N + r) * d;
@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(256) k_compress(const T* __restrict__ x, const
       float v0 = a0 / s0, v1 = a1 / s1;
       if (c >= rope0) {
         float cs, sn;
-        rope_cos_sin(pos, (c - rope0) / 2, rope_dim, theta, &cs, &sn);
+        rope_cos_sin(pos, rope_freq(rope, (c - rope0) / 2), &cs, &sn);
         const float w0 = v0 * cs - v1 * sn, w1 = v0 * sn + v1 * cs;
         v0 = w0;
         v1 = w1;
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) k_compress(const T* __restrict__ x, const
       float2 v = load2(src + c);
       if (c >= rope0) {
         float cs, sn;
-        rope_cos_sin(t, (c - rope0) / 2, rope_dim, theta, &cs, &sn);
+        rope_cos_sin(t, rope_freq(rope, (c - rope0) / 2), &cs, &sn);
         v = make_float2(v.x * cs - v.y * sn, v.x * sn + v.y * cs);
       }
       store2(dst + c, v.x, v.y);

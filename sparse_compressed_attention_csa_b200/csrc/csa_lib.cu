@@ -90,7 +90,37 @@ csa_status_t check_params(const csa_params_t* p) {
   if (p->width < 1 || p->stride < 1)
     return fail(CSA_ERR_INVALID_ARGUMENT, "width=%d stride=%d must be >= 1", p->width, p->stride);
   if (p->window < 0) return fail(CSA_ERR_INVALID_ARGUMENT, "window=%d < 0", p->window);
+  if (!std::isfinite(p->rope_factor))
+    return fail(CSA_ERR_INVALID_ARGUMENT, "rope_factor must be finite");
+  if (p->rope_factor > 1.f &&
+      (p->rope_orig_ctx < 1 || !std::isfinite(p->rope_beta_fast) ||
+       !std::isfinite(p->rope_beta_slow) || !(p->rope_beta_fast > p->rope_beta_slow)))
+    return fail(CSA_ERR_INVALID_ARGUMENT,
+                "YaRN (rope_factor %g > 1) needs rope_orig_ctx >= 1 and rope_beta_fast > "
+                "rope_beta_slow (got %d, %g, %g)",
+                (double)p->rope_factor, p->rope_orig_ctx, (double)p->rope_beta_fast,
+                (double)p->rope_beta_slow);
   return CSA_OK;
+}
+
+// The call's RoPE: plain, or YaRN when rope_factor > 1.
+RopeSpec rope_spec(const csa_params_t* p) {
+  RopeSpec r;
+  r.rope_dim = p->rope_dim;
+  r.theta = (double)p->theta;
+  r.factor = p->rope_factor > 1.f ? (double)p->rope_factor : 1.0;
+  r.orig_ctx = (double)p->rope_orig_ctx;
+  r.beta_fast = (double)p->rope_beta_fast;
+  r.beta_slow = (double)p->rope_beta_slow;
+  return r;
+}
+
+// Softmax scale of the attention calls: `scale`, times YaRN's temperature
+// (0.1 ln s + 1)^2 under the extended RoPE.
+float attn_scale(const csa_params_t* p) {
+  if (!(p->rope_factor > 1.f)) return p->scale;
+  const double m = 0.1 * std::log((double)p->rope_factor) + 1.0;
+  return (float)((double)p->scale * m * m);
 }
 
 csa_status_t check_indexer_shape(const csa_params_t* p) {
@@ -393,12 +423,10 @@ CSA_API csa_status_t csa_compress(const csa_params_t* p, csa_dtype_t dtype, cons
   if (dtype == CSA_BF16)
     k_compress<__nv_bfloat16><<<grid, threads, 0, s>>>(
         (const __nv_bfloat16*)x, (const __nv_bfloat16*)gate, T, p->d, N, p->width, p->stride,
-        p->rope_dim, (double)p->theta, p->pos_offset, (__nv_bfloat16*)kv_cmp_out,
-        (__nv_bfloat16*)kv_raw_rot_out);
+        rope_spec(p), p->pos_offset, (__nv_bfloat16*)kv_cmp_out, (__nv_bfloat16*)kv_raw_rot_out);
   else
     k_compress<float><<<grid, threads, 0, s>>>((const float*)x, (const float*)gate, T, p->d, N,
-                                               p->width, p->stride, p->rope_dim,
-                                               (double)p->theta, p->pos_offset,
+                                               p->width, p->stride, rope_spec(p), p->pos_offset,
                                                (float*)kv_cmp_out, (float*)kv_raw_rot_out);
   return launched("k_compress");
 }
@@ -668,8 +696,7 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
     a.part_o = (__half*)ws;
     a.part_ml = (float*)((char*)ws + o_bytes);
   }
-  for (int i = 0; i < kApMaxRope / 2; ++i)
-    a.freq[i] = i < g.rope_dim / 2 ? std::pow(g.theta, -2.0 * i / (double)g.rope_dim) : 0.0;
+  for (int i = 0; i < kApMaxRope / 2; ++i) a.freq[i] = i < g.rope_dim / 2 ? rope_freq(g.rope, i) : 0.0;
   CUtensorMap tq, to, tc, tr;
   CSA_CHECK(make_tmap_bf16(&tq, g.q, kApDim, (uint64_t)g.B * g.Tq * kApHeads, 64, kApHeads));
   CSA_CHECK(make_tmap_bf16(&to, g.out, kApDim, (uint64_t)g.B * g.Tq * kApHeads, 32, kApHeads,
@@ -713,8 +740,8 @@ static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32
   a.q = q; a.q_pos = q_pos; a.kv_cmp = kv_cmp; a.idx = idx; a.n_cmp = n_cmp; a.n_max = n_max;
   a.kv_raw = kv_raw; a.raw_pos0 = raw_pos0; a.n_raw = n_raw; a.raw_max = raw_max; a.sink = sink;
   a.B = B; a.Tq = Tq; a.H = p->n_heads; a.d = p->d; a.rope_dim = p->rope_dim; a.topk = p->topk;
-  a.window = p->window; a.width = p->width; a.stride = p->stride; a.scale = p->scale;
-  a.theta = (double)p->theta; a.out = out;
+  a.window = p->window; a.width = p->width; a.stride = p->stride; a.scale = attn_scale(p);
+  a.rope = rope_spec(p); a.out = out;
   return a;
 }
 
@@ -853,16 +880,27 @@ CSA_API csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t d
                    kNoAllocScoreFloats * sizeof(float) - sb, s);
 }
 
+static std::atomic<int32_t> g_last_site{0};
+
 CSA_API csa_status_t csa_poll_device_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-  int v = 0;
+  int v = 0, site = 0;
   e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "read device error word");
   if (v == 0) return CSA_OK;
+  e = cudaMemcpyFromSymbol(&site, g_device_error_site, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error site");
+  g_last_site.store(site, std::memory_order_relaxed);
   const int zero = 0;
   e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error_site, &zero, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
-  return fail((csa_status_t)v, "device reported %s", csa_status_string((csa_status_t)v));
+  return fail((csa_status_t)v, "device reported %s (kernel source line %d)",
+              csa_status_string((csa_status_t)v), site);
+}
+
+CSA_API int32_t csa_last_device_error_site(void) {
+  return g_last_site.load(std::memory_order_relaxed);
 }
 

@@ -26,6 +26,7 @@ constexpr int kIdxTcKeys = 128;
 constexpr int kIdxTcHeads = 64;
 constexpr int kIdxTcDim = 128;
 constexpr int kIdxTcThreads = 192;
+constexpr uint64_t kIdxDrainNs = 100000000ull;  // 100 ms for the wind-down waits
 
 template <int QPB, int STAGES>
 struct IdxTcSmem {
@@ -129,10 +130,9 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
         issued = i + 1;
       }
       // drain: every issued copy lands before the CTA may exit
-      int never = 0;
       for (int i = max(0, issued - STAGES); i < issued; ++i)
-        mbar_wait(&sm.full[i % STAGES], (uint32_t)(i / STAGES) & 1u, &never, 100000000ull);
-      mbar_wait(&sm.q_bar, 0, &never, 100000000ull);
+        mbar_drain(&sm.full[i % STAGES], (uint32_t)(i / STAGES) & 1u, kIdxDrainNs);
+      mbar_drain(&sm.q_bar, 0, kIdxDrainNs);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -166,8 +166,7 @@ __global__ void __launch_bounds__(kIdxTcThreads, 1)
         }
       }
       if (last >= 0) {  // the accumulators are released only after the last MMA lands
-        int never = 0;
-        mbar_wait(&sm.acc_full[last & 1], (uint32_t)(last >> 1) & 1u, &never, 100000000ull);
+        mbar_drain(&sm.acc_full[last & 1], (uint32_t)(last >> 1) & 1u, kIdxDrainNs);
       }
     }
   } else {

@@ -12,8 +12,16 @@ namespace sm100 {
 
 // Every wait on an mbarrier gives up after this long, records
 // CSA_ERR_DEVICE_TIMEOUT in the device error word and lets the kernel wind
-// down; a kernel never spins forever.
+// down; a kernel never spins forever.  Once one wait has run out, the
+// launch is failing: every other pipeline wait, in any CTA, gives up at its
+// next clock check instead of running out its own limit, so that a failing
+// launch ends within about one limit rather than one limit per CTA wave.
+// Wind-down drains (copies already in flight into shared memory) do not.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ bool timeout_recorded() {
+  return *reinterpret_cast<volatile int*>(&g_device_error) == CSA_ERR_DEVICE_TIMEOUT;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -72,18 +80,26 @@ __device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity
   return ok != 0;
 }
 
+// A try suspends for at most this long (or the limit, if shorter): a thread
+// wakes as soon as the phase completes anyway, and a short cap keeps the
+// clock checks below frequent, so that a wait that cannot complete runs out
+// close to its limit.
+constexpr uint64_t kMaxSuspendNs = 100000ull;  // 100 us
+
 __device__ __forceinline__ uint32_t suspend_hint(uint64_t limit_ns) {
-  return limit_ns < 0xFFFFFFFFull ? (uint32_t)limit_ns : 0xFFFFFFFFu;
+  return (uint32_t)(limit_ns < kMaxSuspendNs ? limit_ns : kMaxSuspendNs);
 }
 
 // Wait for the phase with the given parity to complete.  Returns false when
-// the CTA is aborting (flag set by another thread) or when this wait ran out
-// (then it sets the flag and records the timeout).  The clock is read after
-// the second unsuccessful try and every 64 tries, and no try suspends longer
-// than the limit, so even a limit of a few nanoseconds runs out on a phase
-// that is not complete at once.
+// the CTA is aborting (flag set by another thread, or a timeout recorded by
+// any CTA) or when this wait ran out (then it sets the flag and records the
+// timeout).  The clock is read after the second unsuccessful try and every
+// 64 tries, and no try suspends longer than the limit, so even a limit of a
+// few nanoseconds runs out on a phase that is not complete at once.  `site`
+// (the caller's source line) is recorded with a timeout.
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                       uint64_t limit_ns = kWaitLimitNs) {
+                                       uint64_t limit_ns = kWaitLimitNs,
+                                       int site = __builtin_LINE()) {
   const uint32_t hint = suspend_hint(limit_ns);
   if (mbar_try_wait_for(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer();
@@ -91,11 +107,32 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
     if (mbar_try_wait_for(bar, parity, hint)) return true;
     if ((it & 63u) == 1u) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > limit_ns) {
+      if (timeout_recorded()) {
         *abort_flag = 1;
-        report_error(CSA_ERR_DEVICE_TIMEOUT);
         return false;
       }
+      if (globaltimer() - t0 > limit_ns) {
+        *abort_flag = 1;
+        report_error(CSA_ERR_DEVICE_TIMEOUT, site);
+        return false;
+      }
+    }
+  }
+}
+
+// Wind-down drain: wait, up to the limit, for a phase that copies already in
+// flight complete.  Only the limit ends it (a failing launch still lets its
+// copies land); running out records the timeout.
+__device__ __noinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                        int site = __builtin_LINE()) {
+  const uint32_t hint = suspend_hint(limit_ns);
+  if (mbar_try_wait_for(bar, parity, hint)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_for(bar, parity, hint)) return true;
+    if ((it & 63u) == 1u && globaltimer() - t0 > limit_ns) {
+      report_error(CSA_ERR_DEVICE_TIMEOUT, site);
+      return false;
     }
   }
 }
@@ -259,7 +296,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 // before the arrival are visible after it).
 __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
                                                volatile int* abort_flag,
-                                               uint64_t limit_ns = kWaitLimitNs) {
+                                               uint64_t limit_ns = kWaitLimitNs,
+                                               int site = __builtin_LINE()) {
   const uint32_t hint = suspend_hint(limit_ns);
   if (mbar_try_wait_cluster(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer();
@@ -267,11 +305,30 @@ __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
     if (mbar_try_wait_cluster(bar, parity, hint)) return true;
     if ((it & 63u) == 1u) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > limit_ns) {
+      if (timeout_recorded()) {
         *abort_flag = 1;
-        report_error(CSA_ERR_DEVICE_TIMEOUT);
         return false;
       }
+      if (globaltimer() - t0 > limit_ns) {
+        *abort_flag = 1;
+        report_error(CSA_ERR_DEVICE_TIMEOUT, site);
+        return false;
+      }
+    }
+  }
+}
+
+// As mbar_drain, for a barrier that other cluster CTAs complete.
+__device__ __noinline__ bool mbar_drain_cluster(uint64_t* bar, uint32_t parity,
+                                                uint64_t limit_ns, int site = __builtin_LINE()) {
+  const uint32_t hint = suspend_hint(limit_ns);
+  if (mbar_try_wait_cluster(bar, parity, hint)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity, hint)) return true;
+    if ((it & 63u) == 1u && globaltimer() - t0 > limit_ns) {
+      report_error(CSA_ERR_DEVICE_TIMEOUT, site);
+      return false;
     }
   }
 }

@@ -4,6 +4,7 @@ call the C ABI.  Every step runs in the CUDA library.
     decode: csa_decode(p, q, q_idx, w, k_idx, kv_cmp, kv_raw, ...) -> (idx, out)
     prefill: csa_prefill(p, x, gate, q_idx, w, k_idx, q, sink) -> (kv_cmp, kv_raw, idx, out)
     HCA decode: hca_decode(p, q, kv_cmp, kv_raw, ...) -> out
+    CSA2 reuse layer: reuse_attn(p, q, ..., kv_cmp, idx, ...) -> out
 """
 from __future__ import annotations
 
@@ -72,4 +73,19 @@ def hca_decode(p: L.Params, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, si
         out = torch.empty_like(q)
     nb = L.csa_workspace_size(p, L.CSA_OP_HCA_ATTN, B, Tq, kv_cmp.shape[1])
     L.hca_attn(p, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, out, ws.get(nb), stream)
+    return out
+
+
+def reuse_attn(p: L.Params, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink,
+               ws: Workspace | None = None, out=None, stream=None):
+    """A Reuse layer of CSA2 ("CSA2 encoder layers (2x compression, Full +
+    Reuse)": the rest reuse that KV and its top-512 selection): this layer's
+    queries and sink over the entries and indices a Full layer produced."""
+    ws = ws or Workspace(q.device)
+    B, Tq = q_pos.shape
+    if out is None:
+        out = torch.empty_like(q)
+    nb = L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, B, Tq, kv_cmp.shape[1])
+    L.csa_sparse_attn(p, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out, ws.get(nb),
+                      stream)
     return out

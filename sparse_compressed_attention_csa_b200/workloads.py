@@ -31,7 +31,8 @@ from dataclasses import dataclass
 
 import numpy as np
 
-_STREAMS = ("x", "g", "k_idx", "q_idx", "w", "q", "sink", "kv_cmp", "kv_raw")
+_STREAMS = ("x", "g", "k_idx", "q_idx", "w", "q", "sink", "kv_cmp", "kv_raw", "q_reuse",
+            "sink_reuse")
 _CHUNK = 1 << 24
 
 
@@ -63,6 +64,11 @@ class Workload:
     pos_offset: int = 0
     int_range: int = 8
     w_exps: tuple = (-2, -1, 0, 1, 2)
+    rope_factor: float = 1.0     # YaRN factor (1: plain RoPE)
+    rope_orig_ctx: int = 0       # YaRN original context
+    rope_beta_fast: float = 32.0
+    rope_beta_slow: float = 1.0
+    reuse_layers: int = 0        # layers attending over this layer's entries and selection
 
     @property
     def scale(self) -> float:
@@ -98,8 +104,25 @@ HCA_DECODE_128K = Workload(
     name="hca_decode_bs16_ctx131072", kind="hca_decode", dtype="bf16", B=16, T=131072, seed=5,
     width=128, stride=128)
 
+# The compressed layers' extended RoPE ("Partial RoPE" rows: theta 160,000
+# with YaRN, factor 16 over 65,536 tokens) on a decode batch whose context
+# (128K tokens) runs past the original 64K.
+CSA_DECODE_YARN = Workload(
+    name="csa_decode_yarn_bs32_ctx131072", kind="csa_decode", dtype="bf16", B=32, T=131072,
+    seed=6, theta=160000.0, rope_factor=16.0, rope_orig_ctx=65536)
+
+# CSA2 ("DeepSeek-V4.1-Flash vs Inkling", row "CSA2 encoder layers (2x
+# compression, Full + Reuse)": KV pooled 2 -> 1 and computed in 3 of 18
+# layers, the rest reuse that KV and its top-512 selection; "Partial RoPE"
+# row: theta 160,000 with YaRN): one Full layer and the 5 Reuse layers that
+# share its entries, on the 64K-context decode batch.
+CSA2_DECODE = Workload(
+    name="csa2_decode_bs32_ctx65536", kind="csa_decode", dtype="bf16", B=32, T=65536, seed=7,
+    width=2, stride=2, topk=512, theta=160000.0, rope_factor=16.0, rope_orig_ctx=65536,
+    reuse_layers=5)
+
 WORKLOADS = {w.name: w for w in (TINY_F32, CSA_DECODE_64K, CSA_PREFILL_8K, CSA_DECODE_1M,
-                                 HCA_DECODE_128K)}
+                                 HCA_DECODE_128K, CSA_DECODE_YARN, CSA2_DECODE)}
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -163,6 +186,7 @@ def generate(wl: Workload, keys=None) -> dict:
     * prefill: x, g [B,T,d] (the caches are produced by pooling in the path)
     * decode kinds: kv_cmp [B,N,d], kv_raw [B,W,d] (already rotated caches),
       raw_pos0 [B], n_raw [B] int32
+    * with reuse layers: q_reuse [R,B,Tq,H,d], sink_reuse [R,H] fp32
     """
     bf16 = wl.dtype == "bf16"
     st = _Streams(wl.seed)
@@ -187,6 +211,10 @@ def generate(wl: Workload, keys=None) -> dict:
         out["n_cmp"] = np.full((B,), N, dtype=np.int32)
     out["q"] = normal(st["q"], (B, Tq, wl.n_heads, d), "q")
     out["sink"] = st["sink"].standard_normal(wl.n_heads, dtype=np.float32)
+    if wl.reuse_layers > 0:
+        R = wl.reuse_layers
+        out["q_reuse"] = normal(st["q_reuse"], (R, B, Tq, wl.n_heads, d), "q_reuse")
+        out["sink_reuse"] = st["sink_reuse"].standard_normal((R, wl.n_heads), dtype=np.float32)
     if wl.kind == "csa_prefill":
         out["q_pos"] = np.tile(np.arange(T, dtype=np.int32), (B, 1))
         out["raw_pos0"] = np.zeros((B,), dtype=np.int32)

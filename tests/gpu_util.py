@@ -27,7 +27,18 @@ def host64(t: torch.Tensor) -> np.ndarray:
 def params_of(wl: Workload) -> Params:
     return Params(d=wl.d, rope_dim=wl.rope_dim, theta=wl.theta, scale=wl.scale,
                   n_heads=wl.n_heads, idx_heads=wl.idx_heads, idx_dim=wl.idx_dim, topk=wl.topk,
-                  window=wl.window, width=wl.width, stride=wl.stride, pos_offset=wl.pos_offset)
+                  window=wl.window, width=wl.width, stride=wl.stride, pos_offset=wl.pos_offset,
+                  rope_factor=wl.rope_factor, rope_orig_ctx=wl.rope_orig_ctx,
+                  rope_beta_fast=wl.rope_beta_fast, rope_beta_slow=wl.rope_beta_slow)
+
+
+def theta_of(wl: Workload):
+    """The oracle's RoPE argument for a workload: the base, or a YaRN spec."""
+    import oracle
+    if wl.rope_factor > 1.0:
+        return oracle.YaRN(theta=wl.theta, factor=wl.rope_factor, orig_ctx=wl.rope_orig_ctx,
+                           beta_fast=wl.rope_beta_fast, beta_slow=wl.rope_beta_slow)
+    return wl.theta
 
 
 def assert_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = ""):

@@ -48,7 +48,7 @@ def test_launch_counter_counts_no_rejected_call(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.csa_abi_version() == 1
+    assert lib.csa_abi_version() == 2
     for code, name in L.STATUS.items():
         assert lib.csa_status_string(code).decode() == name
 
@@ -106,6 +106,12 @@ def test_validation_before_device(lib):
                 dict(stride=0), dict(window=-1), dict(n_heads=0)):
         q = csa.Params(**bad).c()
         assert lib.csa_compress(ctypes.byref(q), 1, P(16), P(16), 1, 64, P(16), None, None) in (1, 3)
+    # extended RoPE (YaRN) without an original context, or with beta_fast <= beta_slow
+    for bad in (dict(rope_factor=16.0, rope_orig_ctx=0),
+                dict(rope_factor=16.0, rope_orig_ctx=65536, rope_beta_fast=1.0, rope_beta_slow=1.0),
+                dict(rope_factor=float("nan"))):
+        q = csa.Params(**bad).c()
+        assert lib.csa_compress(ctypes.byref(q), 1, P(16), P(16), 1, 64, P(16), None, None) == 1
     # topk out of range
     q = csa.Params(topk=0).c()
     assert lib.csa_topk_select(ctypes.byref(q), P(16), P(16), P(16), 1, 1, 10, P(16), None, 0,

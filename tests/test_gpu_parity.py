@@ -12,12 +12,14 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import assert_close, dev, f64, host64, params_of, run_decode, run_hca, run_prefill
+from gpu_util import (assert_close, dev, f64, host64, params_of, run_decode, run_hca,
+                      run_prefill, theta_of)
 from sparse_compressed_attention_csa_b200 import (CSA_OP_SPARSE_ATTN, CSA_OP_TOPK_SELECT,
                                                   CsaError, Params,
                                                   csa_compress, csa_workspace_size,
                                                   csa_index_scores, csa_poll_device_error,
                                                   csa_sparse_attn, csa_topk_select)
+from sparse_compressed_attention_csa_b200 import layer
 from sparse_compressed_attention_csa_b200 import workloads as W
 from sparse_compressed_attention_csa_b200.workloads import bits_to_f32, to_f64
 
@@ -39,7 +41,7 @@ def oracle_decode(wl, data, seqs):
         out = oracle.sparse_attn(f64(data, "q", b), qp, _vals(data["kv_cmp"][b]), idx,
                                  _vals(data["kv_raw"][b]), int(data["raw_pos0"][b]),
                                  int(data["n_raw"][b]), data["sink"], wl.scale, wl.window,
-                                 wl.rope_dim, wl.theta)
+                                 wl.rope_dim, theta_of(wl))
         idx_all.append(idx)
         out_all.append(out)
     return np.stack(idx_all), np.stack(out_all)
@@ -64,7 +66,7 @@ def check_hca(wl, seqs=None):
                                      _vals(data["kv_cmp"][b]), int(data["n_cmp"][b]),
                                      _vals(data["kv_raw"][b]), int(data["raw_pos0"][b]),
                                      int(data["n_raw"][b]), data["sink"], wl.scale, wl.window,
-                                     wl.width, wl.stride, wl.rope_dim, wl.theta)
+                                     wl.width, wl.stride, wl.rope_dim, theta_of(wl))
                      for b in seqs])
     assert_close(got, want, wl.dtype, wl.name)
 
@@ -76,16 +78,16 @@ def check_prefill(wl, rows=None):
     rows = np.arange(T) if rows is None else np.asarray(rows)
     for b in range(wl.B):
         x, g = f64(data, "x", b), f64(data, "g", b)
-        cmp_o = oracle.compress(x, g, wl.width, wl.stride, wl.rope_dim, wl.theta, wl.pos_offset)
+        cmp_o = oracle.compress(x, g, wl.width, wl.stride, wl.rope_dim, theta_of(wl), wl.pos_offset)
         assert_close(host64(kv_cmp[b]), cmp_o, wl.dtype, "compressed entries")
-        raw_o = oracle.rotate_raw(x, 0, wl.rope_dim, wl.theta)
+        raw_o = oracle.rotate_raw(x, 0, wl.rope_dim, theta_of(wl))
         assert_close(host64(kv_raw[b]), raw_o, wl.dtype, "rotated raw rows")
         qp = data["q_pos"][b]
         idx_o = oracle.index_topk(_vals(data["q_idx"][b]), data["w"][b], f64(data, "k_idx", b),
                                   qp, cmp_o.shape[0], wl.width, wl.stride, wl.topk, rows)
         assert np.array_equal(idx[b].cpu().numpy()[rows], idx_o), "top-k indices differ"
         out_o = oracle.sparse_attn(to_f64(data["q"][b][rows]), qp[rows], cmp_o, idx_o, raw_o, 0,
-                                   T, data["sink"], wl.scale, wl.window, wl.rope_dim, wl.theta)
+                                   T, data["sink"], wl.scale, wl.window, wl.rope_dim, theta_of(wl))
         sel = torch.as_tensor(rows, device=out.device)
         assert_close(host64(out[b][sel]), out_o, wl.dtype, wl.name)
 
@@ -122,6 +124,71 @@ def test_decode_ragged_tiles():
 
 def test_decode_fewer_visible_than_k():
     check_decode(W.CSA_DECODE_64K.replace(B=2, T=2100, seed=22))  # N = 524 < 1024
+
+
+def test_decode_running_max_moves_for_some_heads_only():
+    # window row 60 set to 14 x the unit direction of the query of one head
+    # per warp (heads 3, 40, 77, 110; non-rotated dims only): those heads see
+    # a logit of about 13 on it, above their running maximum by more than
+    # the lazy-rescale threshold (2^8), the other heads a small one, so the
+    # lanes of each softmax warp disagree on rescaling O in a late tile.
+    # The row's values stay of order one (the tolerance is absolute).
+    wl = W.CSA_DECODE_64K.replace(B=2, T=5003, seed=47)
+    data = W.generate(wl)
+    raw = bits_to_f32(data["kv_raw"]).copy()
+    q = bits_to_f32(data["q"]).astype(np.float64)  # [B, 1, H, d]
+    nr = wl.d - wl.rope_dim
+    for b in range(wl.B):
+        row = np.zeros(wl.d)
+        for h in (3, 40, 77, 110):
+            u = q[b, 0, h, :nr]
+            row[:nr] += 14.0 * u / np.linalg.norm(u)
+        raw[b, 60] = row
+    data["kv_raw"] = W.bf16_bits(raw)
+    idx, out = run_decode(wl, data)
+    idx_o, out_o = oracle_decode(wl, data, [0, 1])
+    assert np.array_equal(idx.cpu().numpy(), idx_o), "top-k indices differ"
+    assert_close(host64(out), out_o, wl.dtype, "decode with an aligned window row")
+
+
+def test_decode_extended_rope_past_the_original_context():
+    # theta 160,000 with YaRN (factor 16 over 65,536 tokens) on queries at
+    # position 131,071: q and the output's inverse rotation use the YaRN
+    # frequencies, the logits the YaRN temperature
+    check_decode(W.CSA_DECODE_YARN.replace(B=4, seed=44))
+
+
+def test_prefill_extended_rope_small_original_context():
+    # the same extension with an original context of 512 tokens, so that a
+    # 1,500-token prefill runs past it in the pooled entries, the raw rows
+    # and the queries alike; ragged tail, every query row checked
+    wl = W.CSA_PREFILL_8K.replace(T=1500, topk=128, seed=45, theta=160000.0, rope_factor=4.0,
+                                  rope_orig_ctx=512)
+    check_prefill(wl, rows=np.arange(0, 1500, 3))
+
+
+def test_csa2_full_and_reuse_layers():
+    # 2 -> 1 pooling, top-512, YaRN; the Reuse layers attend with their own
+    # queries and sinks over the Full layer's entries and selection
+    wl = W.CSA2_DECODE.replace(B=3, T=20001, reuse_layers=2, seed=46)
+    data = W.generate(wl)
+    idx, out = run_decode(wl, data)
+    seqs = list(range(wl.B))
+    idx_o, out_o = oracle_decode(wl, data, seqs)
+    assert np.array_equal(idx.cpu().numpy(), idx_o), "top-k indices differ"
+    assert_close(host64(out), out_o, wl.dtype, wl.name)
+    p = params_of(wl)
+    t = {k: dev(data[k]) for k in ("q_pos", "kv_cmp", "kv_raw", "raw_pos0", "n_raw")}
+    for r in range(wl.reuse_layers):
+        o = layer.reuse_attn(p, dev(data["q_reuse"][r]), t["q_pos"], t["kv_cmp"], idx,
+                             t["kv_raw"], t["raw_pos0"], t["n_raw"], dev(data["sink_reuse"][r]))
+        torch.cuda.synchronize()
+        want = np.stack([oracle.sparse_attn(
+            f64(data, "q_reuse", r, b),
+            data["q_pos"][b], _vals(data["kv_cmp"][b]), idx_o[b], _vals(data["kv_raw"][b]),
+            int(data["raw_pos0"][b]), int(data["n_raw"][b]), data["sink_reuse"][r], wl.scale,
+            wl.window, wl.rope_dim, theta_of(wl)) for b in seqs])
+        assert_close(host64(o), want, wl.dtype, f"{wl.name} reuse layer {r}")
 
 
 def test_decode_context_too_short_for_any_entry():
@@ -162,7 +229,7 @@ def test_compress_hca_width_bf16_and_f32():
         csa_compress(p, x, g, kv)
         torch.cuda.synchronize()
         want = oracle.compress(f64(data, "x", 0), f64(data, "g", 0), 128, 128, wl.rope_dim,
-                               wl.theta)
+                               theta_of(wl))
         assert_close(host64(kv[0]), want, dtype, f"hca compress {dtype}")
 
 
