@@ -4,6 +4,6 @@ Only `tests/`, `__graft_entry__.smoke()` and `bench.py`'s CPU-baseline legs
 may import this package.  It shares no code with the CUDA path.
 """
 from .csa_oracle import (  # noqa: F401
-    YaRN, attend, attention_temperature, compress, csa_prefill_layer, gather_rows, hca_attn,
-    index_scores, index_topk, n_compressed, n_visible, rope, rope_freqs, rotate_raw, sparse_attn,
-    topk_select, window_tokens)
+    YaRN, attend, attention_temperature, compress, compress_append, csa_prefill_layer,
+    gather_rows, hca_attn, hca_prefill_layer, index_scores, index_topk, n_compressed, n_visible,
+    rope, rope_freqs, rotate_raw, sparse_attn, topk_select, window_tokens)

@@ -197,6 +197,36 @@ def rotate_raw(x: np.ndarray, pos0: int, rope_dim: int, theta) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Step 1 during decode: the entries and raw rows that newly arrived tokens
+# complete ("Compressed Sparse Attention" row: an entry pools tokens
+# stride*j .. stride*j + width - 1, so it exists once its last token has
+# arrived; "Heavily Compressed Attention" row: one entry per 128 tokens)
+# --------------------------------------------------------------------------
+def compress_append(x_win: np.ndarray, g_win: np.ndarray, x_pos0: int, t_old: int, t_new: int,
+                    width: int, stride: int, rope_dim: int, theta, pos_offset: int = 0):
+    """Tokens t_old .. t_new - 1 arrive; x_win[i], g_win[i] are token
+    x_pos0 + i.  The new entries are j0 = N(t_old) .. N(t_new) - 1: the batch
+    compression of the tokens from stride*j0 on, whose positions start at
+    stride*j0.  Returns (j0, entries [N(t_new) - j0, d], raw rows of tokens
+    t_old .. t_new - 1 rotated at their positions)."""
+    x_win = np.asarray(x_win, dtype=np.float64)
+    g_win = np.asarray(g_win, dtype=np.float64)
+    j0 = n_compressed(t_old, width, stride)
+    j1 = n_compressed(t_new, width, stride)
+    lo = stride * j0 - x_pos0 if j1 > j0 else t_old - x_pos0
+    if lo < 0 or t_new - x_pos0 > x_win.shape[0] or t_old - x_pos0 < 0:
+        raise ValueError("the token window does not hold the tokens the new rows need")
+    seg = slice(stride * j0 - x_pos0, t_new - x_pos0)
+    if j1 > j0:
+        ent = compress(x_win[seg], g_win[seg], width, stride, rope_dim, theta,
+                       pos_offset + stride * j0)
+    else:
+        ent = np.zeros((0, x_win.shape[1]), dtype=np.float64)
+    raw = rotate_raw(x_win[t_old - x_pos0:t_new - x_pos0], t_old, rope_dim, theta)
+    return j0, ent, raw
+
+
+# --------------------------------------------------------------------------
 # Step 2: lightning indexer ("64 heads x 128 dims, ReLU scores weighted per
 # head") and top-k ("keeps the top 1,024 entries")
 # --------------------------------------------------------------------------
@@ -328,3 +358,21 @@ def csa_prefill_layer(x, g, q_idx, w, k_idx, q, sink, *, width, stride, topk, wi
     out = sparse_attn(q, q_pos, kv_cmp, full_idx, kv_raw, 0, T, sink, scale, window,
                       rope_dim, theta, rows)
     return kv_cmp, kv_raw, idx, out
+
+
+# --------------------------------------------------------------------------
+# HCA on one prefill sequence ("Heavily Compressed Attention" row: every 128
+# tokens pooled into one entry, dense shared-KV attention over all of them
+# plus a 128-token window), every token a causal query
+# --------------------------------------------------------------------------
+def hca_prefill_layer(x, g, q, sink, *, window, rope_dim, theta, scale, width=128, stride=128,
+                      pos_offset=0, rows=None):
+    """Returns (kv_cmp, kv_raw, out[rows]) for one sequence whose tokens sit
+    at positions 0..T-1: compression, then each query attends to every entry
+    visible to it and its window."""
+    T = np.shape(x)[0]
+    kv_cmp = compress(x, g, width, stride, rope_dim, theta, pos_offset)
+    kv_raw = rotate_raw(x, 0, rope_dim, theta)
+    out = hca_attn(q, np.arange(T), kv_cmp, kv_cmp.shape[0], kv_raw, 0, T, sink, scale, window,
+                   width, stride, rope_dim, theta, rows)
+    return kv_cmp, kv_raw, out

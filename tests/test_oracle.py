@@ -296,6 +296,78 @@ def test_shift_of_all_positions_leaves_output_unchanged():
     np.testing.assert_allclose(outs[2], outs[0], rtol=0, atol=1e-9)
 
 
+# ---------------------------------------------------------------- decode-time append
+@pytest.mark.parametrize("width,stride", [(8, 4), (128, 128), (2, 2), (5, 3)])
+def test_append_equals_batch_compression_in_any_split(width, stride):
+    # token arrivals cut at random points (single tokens, bursts, none): the
+    # appended entries and raw rows, in order, are exactly the batch
+    # compression and rotation of the whole sequence, each entry appearing
+    # once, as soon as its last token has arrived
+    rng = _rng(60 + width)
+    T, d, r = 400, 16, 8
+    x, g = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    full = oracle.compress(x, g, width, stride, r, THETA, pos_offset=3)
+    full_raw = oracle.rotate_raw(x, 0, r, THETA)
+    cuts = np.unique(np.concatenate([[0, T], rng.integers(0, T, 40), np.arange(0, 30)]))
+    ents, raws, seen = [], [], 0
+    for t_old, t_new in zip(cuts[:-1], cuts[1:]):
+        # the window holds just the tokens from the first new entry's start
+        # (or t_old), plus a few before
+        j_first = oracle.n_compressed(int(t_old), width, stride)
+        lo = max(0, min(stride * j_first, int(t_old)) - 3)
+        j0, e, raw = oracle.compress_append(x[lo:t_new], g[lo:t_new], lo, int(t_old), int(t_new),
+                                            width, stride, r, THETA, pos_offset=3)
+        assert j0 == seen
+        for k in range(e.shape[0]):  # entry j exists once its last token has arrived
+            assert stride * (j0 + k) + width - 1 < t_new
+        seen += e.shape[0]
+        ents.append(e)
+        raws.append(raw)
+    assert seen == full.shape[0] == oracle.n_compressed(T, width, stride)
+    np.testing.assert_array_equal(np.concatenate(ents), full)
+    np.testing.assert_array_equal(np.concatenate(raws), full_raw)
+
+
+def test_append_of_one_token_against_brute_force():
+    # the token that completes entry j = 5 (tokens 20..27 at stride 4)
+    # creates exactly that entry, equal to the brute-force pooling of those
+    # taps rotated at position 20
+    rng = _rng(64)
+    x, g = rng.standard_normal((28, 8)), rng.standard_normal((28, 8))
+    j0, e, raw = oracle.compress_append(x[18:], g[18:], 18, 27, 28, 8, 4, 4, THETA)
+    assert j0 == 5 and e.shape[0] == 1
+    ref = brute.compress(x[20:28].tolist(), g[20:28].tolist(), 8, 4, 4, THETA, pos_offset=20)
+    np.testing.assert_allclose(e[0], np.array(ref[0]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(raw[0], np.array(brute._rot(list(x[27]), 27, 4, THETA)),
+                               rtol=0, atol=1e-12)
+    # the tokens before it complete nothing new; a window that lacks a tap fails
+    j0, e, _ = oracle.compress_append(x[18:], g[18:], 18, 25, 27, 8, 4, 4, THETA)
+    assert (j0, e.shape[0]) == (5, 0)
+    with pytest.raises(ValueError):
+        oracle.compress_append(x[21:], g[21:], 21, 27, 28, 8, 4, 4, THETA)
+
+
+# ---------------------------------------------------------------- HCA prefill
+def test_hca_prefill_layer_matches_brute_force():
+    # every token attends to all entries whose 128 tokens it has seen, plus
+    # its window, with the sink; pooling 128 -> 1 without overlap
+    rng = _rng(65)
+    T, d, H, r, W = 300, 8, 2, 4, 16
+    x, g = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    q, sink = rng.standard_normal((T, H, d)), rng.standard_normal(H)
+    rows = np.array([0, 126, 127, 128, 255, 256, 299])
+    kv_cmp, kv_raw, out = oracle.hca_prefill_layer(x, g, q, sink, window=W, rope_dim=r,
+                                                   theta=THETA, scale=0.3, rows=rows)
+    assert kv_cmp.shape[0] == 2
+    b_cmp = brute.compress(x.tolist(), g.tolist(), 128, 128, r, THETA)
+    np.testing.assert_allclose(kv_cmp, np.array(b_cmp), rtol=0, atol=1e-12)
+    for i, t in enumerate(rows):
+        vis = [b_cmp[j] for j in brute.visible(int(t), len(b_cmp), 128, 128)]
+        raw = [brute._rot(list(x[u]), u, r, THETA) for u in brute.window(int(t), W, 0, T)]
+        ref = brute.attend(q[t].tolist(), int(t), vis + raw, sink.tolist(), 0.3, r, THETA)
+        np.testing.assert_allclose(out[i], np.array(ref), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- planted mistakes
 def test_pins_catch_planted_mistakes(monkeypatch):
     """A wrong rotation sign or a dropped sink term in the oracle must trip a pin."""
@@ -323,6 +395,55 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(oracle, "attend", no_sink)
     with pytest.raises(AssertionError):
         test_sink_closed_form_and_weight_sum()
+    monkeypatch.setattr(csa_oracle, "attend", good_attend)
+    monkeypatch.setattr(oracle, "attend", good_attend)
+
+
+def test_pins_catch_half_split_rope(monkeypatch):
+    """RoPE pairs (r0 + i, r0 + i + r/2) instead of the interleaved pairs
+    (r0 + 2i, r0 + 2i + 1) must trip the brute-force and closed-form pins."""
+    good_rope = csa_oracle.rope
+
+    def half_split(x, pos, rope_dim, theta):
+        x = np.asarray(x, dtype=np.float64)
+        r0, h = x.shape[-1] - rope_dim, rope_dim // 2
+        perm = r0 + np.stack([np.arange(h), np.arange(h) + h], axis=1).reshape(-1)
+        y = x.copy()
+        y[..., r0:] = x[..., perm]   # half-split pairs moved to interleaved slots
+        z = good_rope(y, pos, rope_dim, theta)
+        out = z.copy()
+        out[..., perm] = z[..., r0:]
+        return out
+
+    monkeypatch.setattr(csa_oracle, "rope", half_split)
+    monkeypatch.setattr(oracle, "rope", half_split)
+    with pytest.raises(AssertionError):
+        test_rope_is_complex_rotation()
+    with pytest.raises(AssertionError):
+        test_whole_layer_matches_brute_force()
+
+
+def test_pins_catch_transposed_score_matrix(monkeypatch):
+    """Attention weights normalised over the heads instead of over the rows
+    (the query-by-row score matrix used transposed) must trip the SDPA
+    reduction and the brute-force pin."""
+
+    def transposed(q, t, rows, sink, scale, rope_dim, theta):
+        qh = csa_oracle.rope(q, t, rope_dim, theta)
+        rows = np.asarray(rows, dtype=np.float64)
+        z = (rows @ qh.T) * scale * csa_oracle.attention_temperature(theta)  # [R, H]
+        z = np.concatenate([z, np.asarray(sink, dtype=np.float64)[None, :]], axis=0)
+        with np.errstate(invalid="ignore"):  # a sink of -inf: its own row is NaN, dropped
+            e = np.exp(z - z.max(axis=1, keepdims=True))
+        a = (e / e.sum(axis=1, keepdims=True))[:-1]  # rows of a softmax over the heads
+        return csa_oracle.rope(a.T @ rows, -t, rope_dim, theta)
+
+    monkeypatch.setattr(csa_oracle, "attend", transposed)
+    monkeypatch.setattr(oracle, "attend", transposed)
+    with pytest.raises(AssertionError):
+        test_attention_reduces_to_sdpa()
+    with pytest.raises(AssertionError):
+        test_attention_matches_brute_force()
 
 
 # ---------------------------------------------------------------- YaRN
