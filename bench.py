@@ -80,8 +80,8 @@ def _args():
     ap.add_argument("--workload", default=HEADLINE,
                     help="csa_decode_bs32_ctx65536 (default), csa_decode_bs4_ctx1048576, "
                          "hca_decode_bs16_ctx131072, csa_prefill_T8192, "
-                         "csa_decode_yarn_bs32_ctx131072 or csa2_decode_bs32_ctx65536 "
-                         "(one Full + five Reuse layers)")
+                         "csa_decode_yarn_bs32_ctx131072, csa2_decode_bs32_ctx65536 "
+                         "(one Full + five Reuse layers) or hca_prefill_T8192")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--seq-len", type=int, default=0,
@@ -121,7 +121,7 @@ def _config(wl, extra=None, flush_mib=256):
          "l2": (f"flushed before every timed step: {flush_mib} MiB write, then {flush_mib} MiB read "
                 "(L2 left clean)") if flush_mib else "not flushed",
          "parallelism": "replicas"}
-    if wl.kind != "hca_decode":
+    if wl.kind in ("csa_decode", "csa_prefill"):
         c.update({"indexer": f"{wl.idx_heads}x{wl.idx_dim}", "topk": wl.topk})
     if wl.rope_factor > 1.0:
         c["rope"] = (f"theta {wl.theta:g}, YaRN factor {wl.rope_factor:g} over "
@@ -147,6 +147,17 @@ def algorithmic_work(wl):
         g = {"hca_attn": {"bytes": rows + q + out + H * 4,
                           "flops": 4 * n_q * H * (N + wl.window) * d}}
         g["step"] = {"bytes": g["hca_attn"]["bytes"]}
+        return g
+    if wl.kind == "hca_prefill":
+        # causal: query t attends to its visible entries and its window
+        n_rows = sum(max(0, (t - wl.width) // wl.stride + 1) + min(wl.window, t + 1)
+                     for t in range(T))
+        g = {"compress": {"bytes": B * T * d * 2 * 2 + B * N * d * 2 + B * T * d * 2,
+                          "flops": 0},
+             # every entry and raw row read once, q read once, out written once
+             "hca_attn": {"bytes": B * (N + T) * d * 2 + q + out + H * 4,
+                          "flops": 4 * B * H * n_rows * d}}
+        g["step"] = {"bytes": sum(v["bytes"] for v in g.values())}
         return g
     keys = B * N * wl.idx_dim * 2
     idx_q = n_q * wl.idx_heads * (wl.idx_dim * 2 + 4)
@@ -267,6 +278,20 @@ def _oracle_sample(wl):
     th = wl.theta if wl.rope_factor <= 1.0 else oracle.YaRN(
         theta=wl.theta, factor=wl.rope_factor, orig_ctx=wl.rope_orig_ctx,
         beta_fast=wl.rope_beta_fast, beta_slow=wl.rope_beta_slow)
+    if wl.kind == "hca_prefill":
+        data = W.generate(wl)
+        rows = np.linspace(0, wl.T - 1, 16).astype(np.int64)
+
+        def step():
+            kv = oracle.compress(f(data["x"][0]), f(data["g"][0]), wl.width, wl.stride,
+                                 wl.rope_dim, th, wl.pos_offset)
+            raw = oracle.rotate_raw(f(data["x"][0]), 0, wl.rope_dim, th)
+            return oracle.hca_attn(f(data["q"][0][rows]), rows, kv, kv.shape[0], raw, 0, wl.T,
+                                   data["sink"], wl.scale, wl.window, wl.width, wl.stride,
+                                   wl.rope_dim, th)
+        return step, len(rows) * wl.n_heads, (
+            "128 -> 1 compression of the whole sequence, then 128-head attention over every "
+            "visible entry and the window for 16 of the 8,192 query tokens, fp64 NumPy oracle")
     if wl.kind == "csa_prefill":
         data = W.generate(wl)
         rows = np.linspace(0, wl.T - 1, 16).astype(np.int64)
@@ -410,23 +435,26 @@ def run_cuda(args, rank, world, local):
                  rope_beta_fast=wl.rope_beta_fast, rope_beta_slow=wl.rope_beta_slow)
     Bsz, Tq, N = wl.B, wl.Tq, wl.n_cmp
     out = torch.empty_like(t["q"])
-    ops = {"hca_decode": [L.CSA_OP_HCA_ATTN]}.get(
-        wl.kind, [L.CSA_OP_TOPK_SELECT, L.CSA_OP_SPARSE_ATTN])
+    hca = wl.kind in ("hca_decode", "hca_prefill")
+    prefill = wl.kind in ("csa_prefill", "hca_prefill")
+    ops = [L.CSA_OP_HCA_ATTN] if hca else [L.CSA_OP_TOPK_SELECT, L.CSA_OP_SPARSE_ATTN]
     ws = torch.empty(max([L.csa_workspace_size(p, o, Bsz, Tq, N) for o in ops] + [256]),
                      dtype=torch.uint8, device=dev)
-    if wl.kind != "hca_decode":
+    if not hca:
         scores = torch.empty((Bsz, Tq, N), dtype=torch.float32, device=dev)
         idx = torch.empty((Bsz, Tq, wl.topk), dtype=torch.int32, device=dev)
-    if wl.kind == "csa_prefill":
+    if prefill:
         t["kv_cmp"] = torch.empty((Bsz, N, wl.d), dtype=torch.bfloat16, device=dev)
         t["kv_raw"] = torch.empty((Bsz, wl.T, wl.d), dtype=torch.bfloat16, device=dev)
+    if wl.kind == "hca_prefill":
+        t["n_cmp"] = torch.full((Bsz,), N, dtype=torch.int32, device=dev)
 
     # the step's kernel groups, in order
     groups = []
-    if wl.kind == "csa_prefill":
+    if prefill:
         groups.append(("compress", lambda: L.csa_compress(p, t["x"], t["g"], t["kv_cmp"],
                                                           t["kv_raw"])))
-    if wl.kind == "hca_decode":
+    if hca:
         groups.append(("hca_attn", lambda: L.hca_attn(
             p, t["q"], t["q_pos"], t["kv_cmp"], t["n_cmp"], t["kv_raw"], t["raw_pos0"],
             t["n_raw"], t["sink"], out, ws)))
@@ -531,7 +559,8 @@ def run_cuda(args, rank, world, local):
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host
     h2d_keys = {"csa_decode": ("q", "q_idx", "w", "q_pos"), "hca_decode": ("q", "q_pos"),
-                "csa_prefill": ("x", "g", "q_idx", "w", "q")}[wl.kind] + (("q_reuse",) if R else ())
+                "csa_prefill": ("x", "g", "q_idx", "w", "q"),
+                "hca_prefill": ("x", "g", "q")}[wl.kind] + (("q_reuse",) if R else ())
     h_in = {k: torch.from_numpy(np.ascontiguousarray(data[k].view(np.int16) if data[k].dtype ==
                                                       np.uint16 else data[k])).pin_memory()
             for k in h2d_keys}
@@ -568,6 +597,8 @@ def run_cuda(args, rank, world, local):
                 o = layer.hca_decode(p, bf("q"), d_in["q_pos"], t["kv_cmp"], t["n_cmp"],
                                      t["kv_raw"], t["raw_pos0"], t["n_raw"], t["sink"], lw,
                                      out=out)
+            elif wl.kind == "hca_prefill":
+                _, _, o = layer.hca_prefill(p, bf("x"), bf("g"), bf("q"), t["sink"], lw, out=out)
             else:
                 _, _, _, o = layer.csa_prefill(p, bf("x"), bf("g"), bf("q_idx"), d_in["w"],
                                                t["k_idx"], bf("q"), t["sink"], lw)

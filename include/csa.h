@@ -153,6 +153,34 @@ csa_status_t csa_compress(const csa_params_t* p, csa_dtype_t dtype, const void* 
                           const void* gate, int32_t B, int32_t T, void* kv_cmp_out,
                           void* kv_raw_rot_out, void* stream);
 
+/* Step 1 during decode - incremental compression: the entries and rotated
+ * raw rows that the tokens t_old[b] .. t_new[b] - 1 of each sequence
+ * complete, appended to caller-owned caches ("Compressed Sparse Attention"
+ * row: an entry pools tokens s*j .. s*j + width - 1, so it exists once token
+ * s*j + width - 1 has arrived; "Heavily Compressed Attention" row: one entry
+ * per 128 tokens).  Each written value equals what csa_compress writes for
+ * the same tokens.
+ *   x, gate   [B][L][d]  token rows; row i of sequence b is token x_pos0[b] + i
+ *             (a window of the sequence that holds every token the new
+ *             entries pool: from s * n_old back, n_old = entries before
+ *             t_old[b], up to t_new[b] - 1)
+ *   x_pos0, t_old, t_new  [B] int32, device; 0 <= t_new[b] - t_old[b] <= max_new
+ *   kv_cmp    [B][n_cap][d]  entry j at row j; rows n_entries(t_old[b]) ..
+ *             n_entries(t_new[b]) - 1 are written, n_entries(t) =
+ *             floor((t - width)/s) + 1 for t >= width, else 0
+ *   kv_raw    [B][raw_cap][d] (nullable): token t's rotated row at row
+ *             t - raw_pos0[b], for t in t_old[b] .. t_new[b] - 1
+ * max_new (host) bounds the tokens any sequence adds and sizes the launch.
+ * Rows outside these ranges are left untouched.  A sequence whose range
+ * breaks these rules (t_new < t_old, more than max_new tokens) is skipped
+ * whole, a row that needs a token outside x or lands outside its cache is
+ * skipped; both record CSA_ERR_DEVICE_BOUNDS (csa_poll_device_error). */
+csa_status_t csa_compress_append(const csa_params_t* p, csa_dtype_t dtype, const void* x,
+                                 const void* gate, const int32_t* x_pos0, int32_t B, int32_t L,
+                                 const int32_t* t_old, const int32_t* t_new, int32_t max_new,
+                                 void* kv_cmp, int32_t n_cap, void* kv_raw,
+                                 const int32_t* raw_pos0, int32_t raw_cap, void* stream);
+
 /* Step 2a - lightning indexer scores ("64 heads x 128 dims, ReLU scores
  * weighted per head").
  *   q_idx  [B][Tq][H_I][d_I], w [B][Tq][H_I] fp32, k_idx [B][n_max][d_I]

@@ -93,6 +93,8 @@ def _load():
     lib.csa_workspace_size.argtypes = [_PP, ctypes.c_int, _I, _I, _I,
                                        ctypes.POINTER(ctypes.c_size_t)]
     lib.csa_compress.argtypes = [_PP, ctypes.c_int, _P, _P, _I, _I, _P, _P, _P]
+    lib.csa_compress_append.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _I, _I, _P, _P, _I, _P, _I,
+                                        _P, _P, _I, _P]
     lib.csa_index_scores.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]
     lib.csa_topk_select.argtypes = [_PP, _P, _P, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]
     lib.csa_index_topk.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P,
@@ -111,6 +113,7 @@ def _load():
     lib.csa_last_device_error_site.argtypes = []
     for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
               "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error",
+              "csa_compress_append",
               "csa_index_topk_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -177,6 +180,28 @@ def csa_compress(p: Params, x, gate, kv_cmp_out, kv_raw_rot_out=None, stream=Non
     B, T, d = x.shape
     _check(_load().csa_compress(ctypes.byref(p.c()), _dtype_code(x), _ptr(x), _ptr(gate), B, T,
                                 _ptr(kv_cmp_out), _ptr(kv_raw_rot_out), _stream(stream)))
+
+
+def csa_compress_append(p: Params, x, gate, x_pos0, t_old, t_new, max_new: int, kv_cmp,
+                        kv_raw=None, raw_pos0=None, stream=None):
+    """Entries and raw rows completed by tokens t_old[b] .. t_new[b] - 1:
+    x, gate [B][L][d] (row i = token x_pos0[b] + i) -> rows of kv_cmp
+    [B][n_cap][d] (entry j at row j) and kv_raw [B][raw_cap][d] (token t at
+    row t - raw_pos0[b])."""
+    import torch
+    _req(x, "x", ndim=3)
+    _req(gate, "gate", x.dtype, 3)
+    for t, n in ((x_pos0, "x_pos0"), (t_old, "t_old"), (t_new, "t_new")):
+        _req(t, n, torch.int32, 1)
+    _req(kv_cmp, "kv_cmp", x.dtype, 3)
+    if kv_raw is not None:
+        _req(kv_raw, "kv_raw", x.dtype, 3)
+        _req(raw_pos0, "raw_pos0", torch.int32, 1)
+    B, L, d = x.shape
+    _check(_load().csa_compress_append(
+        ctypes.byref(p.c()), _dtype_code(x), _ptr(x), _ptr(gate), _ptr(x_pos0), B, L, _ptr(t_old),
+        _ptr(t_new), int(max_new), _ptr(kv_cmp), kv_cmp.shape[1], _ptr(kv_raw),
+        _ptr(raw_pos0), kv_raw.shape[1] if kv_raw is not None else 0, _stream(stream)))
 
 
 def csa_index_scores(p: Params, q_idx, w, k_idx, q_pos, n_cmp, scores, stream=None):

@@ -162,16 +162,6 @@ __device__ __forceinline__ uint32_t ap_swz64(int r, int u) {
   return (uint32_t)(r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
 }
 
-// cos / sin of pos * freq: the angle is reduced modulo 2 pi in double
-// precision (2 pi split in two parts), then taken in fp32.
-__device__ __forceinline__ void ap_rope_cs(long long pos, double freq, float* c, float* s) {
-  const double x = (double)pos * freq;
-  const double k = rint(x * 0.15915494309189535);
-  double r = fma(-k, 6.283185307179586, x);
-  r = fma(-k, 2.4492935982947064e-16, r);
-  sincosf((float)r, s, c);
-}
-
 // All 128 threads of warps 0-3 agree on `ok` (named barrier 1).
 __device__ __forceinline__ bool ap_softmax_all(bool ok) {
   uint32_t all;
@@ -262,7 +252,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
     // RoPE table at the query position
     for (int i = lane; i < a.rope_dim / 2; i += 32) {
       float c, s;
-      ap_rope_cs(t, a.freq[i], &c, &s);
+      rope_cs_reduced(t, a.freq[i], &c, &s);
       sm.cs[i] = c;
       sm.sn[i] = s;
     }
@@ -861,7 +851,7 @@ __global__ void __launch_bounds__(kApHeads) k_attn_merge(AttnMergeArgs a) {
     const int d = d0 + 2 * head;
     if (d >= rope0) {
       float c, s;
-      ap_rope_cs(a.q_pos[row_q], a.freq[(d - rope0) >> 1], &c, &s);
+      rope_cs_reduced(a.q_pos[row_q], a.freq[(d - rope0) >> 1], &c, &s);
       cs[head] = c;
       sn[head] = s;
     }

@@ -74,6 +74,20 @@ __device__ __forceinline__ void rope_cos_sin(long long pos, double freq, float* 
   *s = (float)sd;
 }
 
+// cos / sin of pos * freq for the tensor-core and streaming kernels: the
+// angle is formed in double precision and reduced modulo 2 pi there (2 pi
+// split into a double and its remainder, a Cody-Waite reduction), and the
+// reduced angle, in [-pi, pi], goes to the hardware sine / cosine (absolute
+// error about 5e-7 on that range).  The angle's own error stays near 1e-16
+// of pos * freq, so positions up to 2^20 lose nothing more.
+__device__ __forceinline__ void rope_cs_reduced(long long pos, double freq, float* c, float* s) {
+  const double x = (double)pos * freq;
+  const double k = rint(x * 0.15915494309189535);
+  double r = fma(-k, 6.283185307179586, x);
+  r = fma(-k, 2.4492935982947064e-16, r);
+  __sincosf((float)r, s, c);
+}
+
 // Entries j < n_cmp whose last pooled token s*j + w - 1 is at most t.
 __device__ __forceinline__ int n_visible(int t, int n_cmp, int width, int stride) {
   if (t < width - 1) return 0;

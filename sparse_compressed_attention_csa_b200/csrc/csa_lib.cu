@@ -402,6 +402,43 @@ CSA_API csa_status_t csa_workspace_size(const csa_params_t* p, csa_op_t op, int3
   return fail(CSA_ERR_INVALID_ARGUMENT, "bad op %d", (int)op);
 }
 
+// e_slots: entries per sequence the launch covers; a.n_raw: raw rows.
+static csa_status_t launch_compress(CompressArgs& a, int e_slots, csa_dtype_t dtype, int B,
+                                    cudaStream_t s) {
+  if (a.rope.rope_dim / 2 > kCompressMaxPairs)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "rope_dim=%d", a.rope.rope_dim);
+  for (int i = 0; i < kCompressMaxPairs; ++i)
+    a.freq[i] = i < a.rope.rope_dim / 2 ? rope_freq(a.rope, i) : 0.0;
+  const bool wide = a.width >= kCompressWideMin;
+  a.wide_ctas = wide ? e_slots : 0;
+  a.narrow_slots = wide ? 0 : e_slots;
+  a.raw_slots = (a.n_raw + kCompressRawPer - 1) / kCompressRawPer;
+  const int vec = dtype == CSA_BF16 ? 8 : 4;
+  const int rpc = kCompressThreads / (a.d / vec);
+  const long long ctas =
+      a.wide_ctas + ((long long)a.narrow_slots + a.raw_slots + rpc - 1) / rpc;
+  if (ctas == 0) return CSA_OK;
+  if (ctas > 2147483647LL) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "too many rows");
+  dim3 grid((unsigned)ctas, (unsigned)B);
+  if (dtype == CSA_BF16)
+    k_compress<__nv_bfloat16><<<grid, kCompressThreads, 0, s>>>(a);
+  else
+    k_compress<float><<<grid, kCompressThreads, 0, s>>>(a);
+  return launched("k_compress");
+}
+
+static CompressArgs compress_args(const csa_params_t* p, const void* x, const void* gate) {
+  CompressArgs a{};
+  a.x = x;
+  a.g = gate;
+  a.d = p->d;
+  a.width = p->width;
+  a.stride = p->stride;
+  a.pos_offset = p->pos_offset;
+  a.rope = rope_spec(p);
+  return a;
+}
+
 CSA_API csa_status_t csa_compress(const csa_params_t* p, csa_dtype_t dtype, const void* x,
                           const void* gate, int32_t B, int32_t T, void* kv_cmp_out,
                           void* kv_raw_rot_out, void* stream) {
@@ -414,21 +451,54 @@ CSA_API csa_status_t csa_compress(const csa_params_t* p, csa_dtype_t dtype, cons
   const int N = T < p->width ? 0 : (T - p->width) / p->stride + 1;
   if (N > 0) CSA_CHECK(check_ptr(kv_cmp_out, "kv_cmp_out"));
   CSA_CHECK(check_device());
-  const long long rows = (long long)N + (kv_raw_rot_out ? T : 0);
-  if (rows == 0) return CSA_OK;
-  if (rows > 2147483647LL) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "too many rows");
-  cudaStream_t s = (cudaStream_t)stream;
-  dim3 grid((unsigned)rows, (unsigned)B);
-  const int threads = p->d / 2 < 256 ? p->d / 2 : 256;
-  if (dtype == CSA_BF16)
-    k_compress<__nv_bfloat16><<<grid, threads, 0, s>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)gate, T, p->d, N, p->width, p->stride,
-        rope_spec(p), p->pos_offset, (__nv_bfloat16*)kv_cmp_out, (__nv_bfloat16*)kv_raw_rot_out);
-  else
-    k_compress<float><<<grid, threads, 0, s>>>((const float*)x, (const float*)gate, T, p->d, N,
-                                               p->width, p->stride, rope_spec(p), p->pos_offset,
-                                               (float*)kv_cmp_out, (float*)kv_raw_rot_out);
-  return launched("k_compress");
+  CompressArgs a = compress_args(p, x, gate);
+  a.L = T;
+  a.T = T;
+  a.max_new = T;
+  a.n_raw = kv_raw_rot_out ? T : 0;
+  a.kv_cmp = kv_cmp_out;
+  a.n_cap = N;
+  a.kv_raw = kv_raw_rot_out;
+  a.raw_cap = T;
+  return launch_compress(a, N, dtype, B, (cudaStream_t)stream);
+}
+
+CSA_API csa_status_t csa_compress_append(const csa_params_t* p, csa_dtype_t dtype, const void* x,
+                                         const void* gate, const int32_t* x_pos0, int32_t B,
+                                         int32_t L, const int32_t* t_old, const int32_t* t_new,
+                                         int32_t max_new, void* kv_cmp, int32_t n_cap,
+                                         void* kv_raw, const int32_t* raw_pos0, int32_t raw_cap,
+                                         void* stream) {
+  CSA_CHECK(check_params(p));
+  CSA_CHECK(check_dtype(dtype));
+  if (B < 1 || B > 65535 || L < 0 || max_new < 0 || n_cap < 0 || raw_cap < 0)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "B=%d L=%d max_new=%d n_cap=%d raw_cap=%d", B, L,
+                max_new, n_cap, raw_cap);
+  CSA_CHECK(check_ptr(x, "x", L == 0));
+  CSA_CHECK(check_ptr(gate, "gate", L == 0));
+  CSA_CHECK(check_ptr(x_pos0, "x_pos0"));
+  CSA_CHECK(check_ptr(t_old, "t_old"));
+  CSA_CHECK(check_ptr(t_new, "t_new"));
+  CSA_CHECK(check_ptr(kv_cmp, "kv_cmp", n_cap == 0));
+  CSA_CHECK(check_ptr(kv_raw, "kv_raw", true));
+  if (kv_raw) CSA_CHECK(check_ptr(raw_pos0, "raw_pos0"));
+  CSA_CHECK(check_device());
+  CompressArgs a = compress_args(p, x, gate);
+  a.x_pos0 = x_pos0;
+  a.L = L;
+  a.t_old = t_old;
+  a.t_new = t_new;
+  a.max_new = max_new;
+  // entries completed by max_new consecutive tokens: at most ceil(max_new / stride)
+  int e_slots = (int)(((long long)max_new + p->stride - 1) / p->stride);
+  a.n_raw = kv_raw ? max_new : 0;
+  if (e_slots + a.n_raw == 0) e_slots = 1;  // one CTA still checks t_new - t_old
+  a.kv_cmp = kv_cmp;
+  a.n_cap = n_cap;
+  a.kv_raw = kv_raw;
+  a.raw_pos0 = raw_pos0;
+  a.raw_cap = raw_cap;
+  return launch_compress(a, e_slots, dtype, B, (cudaStream_t)stream);
 }
 
 template <int QPB, int STAGES>

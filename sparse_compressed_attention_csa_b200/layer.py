@@ -4,7 +4,9 @@ call the C ABI.  Every step runs in the CUDA library.
     decode: csa_decode(p, q, q_idx, w, k_idx, kv_cmp, kv_raw, ...) -> (idx, out)
     prefill: csa_prefill(p, x, gate, q_idx, w, k_idx, q, sink) -> (kv_cmp, kv_raw, idx, out)
     HCA decode: hca_decode(p, q, kv_cmp, kv_raw, ...) -> out
+    HCA prefill: hca_prefill(p, x, gate, q, sink) -> (kv_cmp, kv_raw, out)
     CSA2 reuse layer: reuse_attn(p, q, ..., kv_cmp, idx, ...) -> out
+    decode-time append: append_tokens(p, x, gate, x_pos0, t_old, t_new, ...)
 """
 from __future__ import annotations
 
@@ -89,3 +91,34 @@ def reuse_attn(p: L.Params, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink
     L.csa_sparse_attn(p, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out, ws.get(nb),
                       stream)
     return out
+
+
+def hca_prefill(p: L.Params, x, gate, q, sink, ws: Workspace | None = None, out=None,
+                stream=None):
+    """HCA on B sequences of T tokens, every token a causal query ("Heavily
+    Compressed Attention" row: every 128 tokens pooled into one entry, dense
+    attention over all of them plus a 128-token window); p.width and
+    p.stride give the pooling."""
+    ws = ws or Workspace(x.device)
+    B, T, d = x.shape
+    N = 0 if T < p.width else (T - p.width) // p.stride + 1
+    dev = x.device
+    kv_cmp = torch.empty((B, N, d), dtype=x.dtype, device=dev)
+    kv_raw = torch.empty((B, T, d), dtype=x.dtype, device=dev)
+    L.csa_compress(p, x, gate, kv_cmp, kv_raw, stream)
+    q_pos = torch.arange(T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+    n_cmp = torch.full((B,), N, dtype=torch.int32, device=dev)
+    raw_pos0 = torch.zeros((B,), dtype=torch.int32, device=dev)
+    out = hca_decode(p, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_cmp.new_full((B,), T), sink,
+                     ws, out, stream)
+    return kv_cmp, kv_raw, out
+
+
+def append_tokens(p: L.Params, x, gate, x_pos0, t_old, t_new, max_new: int, kv_cmp,
+                  kv_raw=None, raw_pos0=None, stream=None):
+    """Decode-time compression: write the entries and rotated raw rows that
+    tokens t_old[b] .. t_new[b] - 1 complete into the caches (entry j at
+    row j of kv_cmp, token t at row t - raw_pos0[b] of kv_raw); x, gate hold
+    token x_pos0[b] + i at row i."""
+    L.csa_compress_append(p, x, gate, x_pos0, t_old, t_new, max_new, kv_cmp, kv_raw, raw_pos0,
+                          stream)

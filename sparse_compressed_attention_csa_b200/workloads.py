@@ -42,7 +42,7 @@ class Workload:
 
     kind: "csa_decode" (pre-compressed caches, one query per sequence),
           "csa_prefill" (token KV + gates are pooled in the path, every
-          token is a causal query) or "hca_decode".
+          token is a causal query), "hca_decode" or "hca_prefill".
     """
 
     name: str
@@ -83,7 +83,7 @@ class Workload:
 
     @property
     def Tq(self) -> int:
-        return self.T if self.kind == "csa_prefill" else 1
+        return self.T if self.kind in ("csa_prefill", "hca_prefill") else 1
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -121,8 +121,16 @@ CSA2_DECODE = Workload(
     width=2, stride=2, topk=512, theta=160000.0, rope_factor=16.0, rope_orig_ctx=65536,
     reuse_layers=5)
 
+# HCA on a prefill sequence ("Heavily Compressed Attention" row: 128 tokens
+# -> 1 entry, dense attention over every entry plus the window), the CSA
+# prefill's length: 64 entries, every token a causal query.
+HCA_PREFILL_8K = Workload(
+    name="hca_prefill_T8192", kind="hca_prefill", dtype="bf16", B=1, T=8192, seed=8,
+    width=128, stride=128)
+
 WORKLOADS = {w.name: w for w in (TINY_F32, CSA_DECODE_64K, CSA_PREFILL_8K, CSA_DECODE_1M,
-                                 HCA_DECODE_128K, CSA_DECODE_YARN, CSA2_DECODE)}
+                                 HCA_DECODE_128K, CSA_DECODE_YARN, CSA2_DECODE,
+                                 HCA_PREFILL_8K)}
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -200,7 +208,8 @@ def generate(wl: Workload, keys=None) -> dict:
     def ints(rng, shape, key):
         return _ints(rng, shape, wl.int_range, bf16) if want(key) else None
 
-    if wl.kind == "csa_prefill":
+    prefill = wl.kind in ("csa_prefill", "hca_prefill")
+    if prefill:
         out["x"] = normal(st["x"], (B, T, d), "x")
         out["g"] = normal(st["g"], (B, T, d), "g")
     if wl.kind in ("csa_prefill", "csa_decode"):
@@ -215,7 +224,7 @@ def generate(wl: Workload, keys=None) -> dict:
         R = wl.reuse_layers
         out["q_reuse"] = normal(st["q_reuse"], (R, B, Tq, wl.n_heads, d), "q_reuse")
         out["sink_reuse"] = st["sink_reuse"].standard_normal((R, wl.n_heads), dtype=np.float32)
-    if wl.kind == "csa_prefill":
+    if prefill:
         out["q_pos"] = np.tile(np.arange(T, dtype=np.int32), (B, 1))
         out["raw_pos0"] = np.zeros((B,), dtype=np.int32)
         out["n_raw"] = np.full((B,), T, dtype=np.int32)

@@ -92,6 +92,29 @@ def check_prefill(wl, rows=None):
         assert_close(host64(out[b][sel]), out_o, wl.dtype, wl.name)
 
 
+def check_hca_prefill(wl, rows=None):
+    data = W.generate(wl)
+    p = params_of(wl)
+    kv_cmp, kv_raw, out = layer.hca_prefill(p, dev(data["x"]), dev(data["g"]), dev(data["q"]),
+                                            dev(data["sink"]))
+    torch.cuda.synchronize()
+    T = wl.T
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    th = theta_of(wl)
+    for b in range(wl.B):
+        x, g = f64(data, "x", b), f64(data, "g", b)
+        cmp_o = oracle.compress(x, g, wl.width, wl.stride, wl.rope_dim, th, wl.pos_offset)
+        assert_close(host64(kv_cmp[b]), cmp_o, wl.dtype, "HCA entries")
+        raw_o = oracle.rotate_raw(x, 0, wl.rope_dim, th)
+        assert_close(host64(kv_raw[b]), raw_o, wl.dtype, "HCA raw rows")
+        # the oracle's HCA prefill restricted to the sampled query rows
+        out_o = oracle.hca_attn(to_f64(data["q"][b][rows]), rows, cmp_o, cmp_o.shape[0], raw_o,
+                                0, T, data["sink"], wl.scale, wl.window, wl.width, wl.stride,
+                                wl.rope_dim, th)
+        sel = torch.as_tensor(rows, device=out.device)
+        assert_close(host64(out[b][sel]), out_o, wl.dtype, wl.name)
+
+
 # ------------------------------------------------------------------ the five workloads
 def test_tiny_f32_full_layer():
     check_prefill(W.TINY_F32)
@@ -117,6 +140,18 @@ def test_csa_prefill_8k():
 
 
 # ------------------------------------------------------------------ smaller cases
+def test_hca_prefill_8k():
+    # every entry and raw row; query rows: the first 300 (0, 1 and 2 entries
+    # visible, the window filling up) and a stride through the rest
+    rows = np.unique(np.concatenate([np.arange(300), np.arange(300, 8192, 37), [8191]]))
+    check_hca_prefill(W.HCA_PREFILL_8K, rows)
+
+
+def test_hca_prefill_ragged_small():
+    # T = 1000: 7 entries, a partial last block of 104 tokens; two sequences
+    check_hca_prefill(W.HCA_PREFILL_8K.replace(B=2, T=1000, seed=48))
+
+
 def test_decode_ragged_tiles():
     # N = 1249 (ragged), selection active (n_vis > k), raw window 128
     check_decode(W.CSA_DECODE_64K.replace(B=3, T=5003, seed=21))
