@@ -282,8 +282,38 @@ struct TopkPlan {
   int chunks;     // 0: generic; 1: single stage; >1: chunk + merge
   int chunk_len;  // entries per chunk block
   int merge_cap;  // candidates per merge block
-  int cluster;    // > 1: one cluster of this many 4096-entry CTAs per row
+  int cluster;    // > 1: one cluster of this many CTAs per row, of chunk_len entries each
 };
+
+// Whether a cluster of `c` 1024-thread top-k CTAs (a non-portable size
+// above 8) can be resident on this device; asked once per device and size.
+static bool wide_topk_cluster_fits(int c) {
+  static signed char known[64][kTopkMaxWideCluster + 1];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || c < 2 || c > kTopkMaxWideCluster) return false;
+  if (known[dev][c]) return known[dev][c] > 0;
+  auto kern = k_topk_cluster<1024, 16, kTopkMaxWideCluster>;
+  bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)c, 1);
+    cfg.blockDim = dim3(1024);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)c;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    ok = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0;
+  }
+  cudaGetLastError();  // a refusal above is an answer, not an error to keep
+  known[dev][c] = ok ? 1 : -1;
+  return ok;
+}
 constexpr int kTopkSmall = 256 * 8, kTopkMid = 256 * 16, kTopkBig = 1024 * 16;
 
 TopkPlan topk_plan(const csa_params_t* p, int B, int Tq, int n_max) {
@@ -293,6 +323,11 @@ TopkPlan topk_plan(const csa_params_t* p, int B, int Tq, int n_max) {
   if (n_max > kTopkMid && n_max <= kTopkMaxCluster * kTopkMid && 2 * rows <= num_sms()) {
     const int c = (n_max + kTopkMid - 1) / kTopkMid;
     if (rows * c <= num_sms()) return {1, kTopkMid, 0, c};
+  }
+  // few very long rows: a cluster of up to 16 CTAs of 16,384 entries per row
+  if (n_max > kTopkMaxCluster * kTopkMid && n_max <= kTopkMaxWideCluster * kTopkBig) {
+    const int c = (n_max + kTopkBig - 1) / kTopkBig;
+    if (rows * c <= num_sms() && wide_topk_cluster_fits(c)) return {1, kTopkBig, 0, c};
   }
   if (n_max <= kTopkSmall) return {1, kTopkSmall, 0, 0};
   if (n_max <= kTopkBig) return {1, kTopkBig, 0, 0};
@@ -577,8 +612,13 @@ static csa_status_t topk_impl(const csa_params_t* p, const float* scores, const 
   int* none = nullptr;
   if (plan.cluster > 1) {
     const cudaError_t e =
-        launch_ex(k_topk_cluster<256, 16>, dim3((unsigned)plan.cluster, rows), dim3(256), 0, s,
-                  plan.cluster, scores, q_pos, n_cmp, Tq, n_max, k, p->width, p->stride, idx_out);
+        plan.chunk_len == kTopkMid
+            ? launch_ex(k_topk_cluster<256, 16>, dim3((unsigned)plan.cluster, rows), dim3(256), 0,
+                        s, plan.cluster, scores, q_pos, n_cmp, Tq, n_max, k, p->width, p->stride,
+                        idx_out)
+            : launch_ex(k_topk_cluster<1024, 16, kTopkMaxWideCluster>,
+                        dim3((unsigned)plan.cluster, rows), dim3(1024), 0, s, plan.cluster, scores,
+                        q_pos, n_cmp, Tq, n_max, k, p->width, p->stride, idx_out);
     if (e != cudaSuccess) return cuda_fail(e, "k_topk_cluster");
     return launched("k_topk_cluster");
   }

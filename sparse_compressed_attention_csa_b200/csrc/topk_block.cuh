@@ -284,20 +284,22 @@ __global__ void __launch_bounds__(NT)
 
 // ---------------------------------------------------------------------------
 // Few long rows: one thread-block cluster of C CTAs per row (C = gridDim.x,
-// at most kTopkMaxCluster), CTA c holding entries [c * NT * PT, (c + 1) * NT
-// * PT) striped as above.  The CTAs exchange, through distributed shared
+// at most MAXC: up to 8 CTAs of 4,096 entries, or up to 16 of 16,384 for
+// rows of up to 262,144 entries), CTA c holding entries [c * NT * PT,
+// (c + 1) * NT * PT) striped as above.  The CTAs exchange, through distributed shared
 // memory, their valid counts and AND/OR of keys, each radix pass's 256-bin
 // histogram and, at the end, their counts of greater and boundary keys; one
 // cluster barrier per exchange.  Every CTA then takes the same decisions on
 // the same totals and places its kept entries after those of the lower
 // ranks, so the row's output is the single-block result.
-constexpr int kTopkMaxCluster = 8;
+constexpr int kTopkMaxCluster = 8;       // 4,096-entry CTAs (256 x 16), portable cluster
+constexpr int kTopkMaxWideCluster = 16;  // 16,384-entry CTAs (1024 x 16), non-portable size
 
-template <int NT, int PT>
+template <int NT, int PT, int MAXC>
 struct TopkClusterShared {
   TopkShared<NT, PT> loc;
-  unsigned xh[2][kTopkMaxCluster][256];  // per-pass histograms of every rank (double buffer)
-  int xv[3][kTopkMaxCluster][3];         // small per-rank values of the three exchanges
+  unsigned xh[2][MAXC][256];  // per-pass histograms of every rank (double buffer)
+  int xv[3][MAXC][3];         // small per-rank values of the three exchanges
 };
 
 // Stores v at the same shared-memory offset as `local` in cluster CTA `rank`.
@@ -309,14 +311,15 @@ __device__ __forceinline__ void dsmem_store(const void* local, uint32_t rank, ui
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
 }
 
-template <int NT, int PT>
+template <int NT, int PT, int MAXC = kTopkMaxCluster>
 __global__ void __launch_bounds__(NT)
     k_topk_cluster(const float* __restrict__ scores, const int* __restrict__ q_pos,
                    const int* __restrict__ n_cmp, int Tq, int n_max, int k, int width,
                    int stride, int* __restrict__ idx_out) {
   static_assert(NT >= 256, "bin scan needs 256 threads");
+  static_assert(NT * PT < 65536, "per-CTA counts are packed in 16 bits");
   constexpr int NW = NT / 32;
-  __shared__ TopkClusterShared<NT, PT> sh;
+  __shared__ TopkClusterShared<NT, PT, MAXC> sh;
   sm100::griddep_wait();  // the scores of the predecessor are visible
   sm100::griddep_launch_dependents();
   const int C = (int)gridDim.x;

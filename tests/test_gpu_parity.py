@@ -316,9 +316,9 @@ def _adversarial_rows(rng, n):
 
 
 # (entries, k, rows, visible): few rows of up to 32768 entries take a cluster
-# of 4096-entry CTAs per row; otherwise one block per row up to 16384
-# entries, else chunks of 16384 and a merge block of 4096, 8192 or 16384
-# candidates
+# of 4096-entry CTAs per row, few rows of up to 262144 a cluster of up to 16
+# CTAs of 16384; otherwise one block per row up to 16384 entries, else
+# chunks of 16384 and a merge block of 4096, 8192 or 16384 candidates
 @pytest.mark.parametrize("n,k,rows,visible", [
     (5000, 1024, 7, None),     # cluster of 2
     (9000, 64, 3, None),       # cluster of 3
@@ -327,9 +327,12 @@ def _adversarial_rows(rng, n):
     (20000, 1024, 3, 700),     # cluster of 5, fewer visible than k
     (5000, 1024, 84, None),    # one 16384-entry block per row
     (1500, 64, 20, None),      # one 2048-entry block per row
-    (40000, 1024, 7, None),    # 3 chunks, merge of 3072 candidates
-    (70000, 1024, 7, None),    # 5 chunks, merge of 5120
-    (70000, 3000, 3, None),    # 5 chunks, merge of 15000
+    (40000, 1024, 7, None),    # cluster of 3 CTAs of 16384 entries
+    (70000, 3000, 3, None),    # cluster of 5 of 16384, k = 3000
+    (262143, 1024, 4, None),   # cluster of 16 of 16384 (the 1M-context rows)
+    (200000, 1024, 3, 150001), # cluster of 13, fewer visible than the CTAs hold
+    (40000, 1024, 60, None),   # 180 CTAs for a cluster each: 3 chunks, merge of 3072
+    (70000, 1024, 40, None),   # 5 chunks, merge of 5120
 ])
 def test_topk_select_adversarial_scores(n, k, rows, visible):
     rng = np.random.default_rng(29 + n + k + rows)
