@@ -227,6 +227,61 @@ def compress_append(x_win: np.ndarray, g_win: np.ndarray, x_pos0: int, t_old: in
 
 
 # --------------------------------------------------------------------------
+# KV cache quantized after RoPE ("DeepSeek-V4.1-Flash vs Inkling", "Partial
+# RoPE" row: the KV cache is quantized after RoPE; the pages give no
+# format).  Read here as 8-bit floats E4M3 of the OCP 8-bit floating point
+# specification (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
+# no infinities, S.1111.111 the only NaN, largest finite 448) with one fp32
+# scale per cache row: scale = max|row| / 448 (1 for an all-zero row), code
+# = the E4M3 value nearest to x / scale, ties to the even code, magnitudes
+# above 448 saturated.  The division and the scale are taken in fp32, the
+# precision the codes are decided in on the GPU.
+# --------------------------------------------------------------------------
+def e4m3_values() -> np.ndarray:
+    """The value of each of the 256 E4M3 codes (NaN for the two NaN codes)."""
+    vals = np.empty(256, dtype=np.float64)
+    for c in range(256):
+        sign = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 0xF, c & 0x7
+        if e == 0xF and m == 0x7:
+            vals[c] = np.nan
+        elif e == 0:
+            vals[c] = sign * 2.0 ** -6 * (m / 8.0)           # subnormal
+        else:
+            vals[c] = sign * 2.0 ** (e - 7) * (1.0 + m / 8.0)
+    return vals
+
+
+def e4m3_encode(y: np.ndarray) -> np.ndarray:
+    """Round each (finite) value to the nearest E4M3 code, ties to the even
+    code, saturating at +-448; the sign of zero is kept."""
+    y = np.asarray(y, dtype=np.float64)
+    pos = e4m3_values()[:127]               # codes 0..126: 0, subnormals, normals to 448
+    a = np.minimum(np.abs(y), pos[-1])
+    hi = np.clip(np.searchsorted(pos, a, side="left"), 0, 126)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - pos[lo], pos[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return np.where(np.signbit(y), code | np.uint8(0x80), code).astype(np.uint8)
+
+
+def quantize_fp8_rows(rows: np.ndarray):
+    """Cache rows [n, d] (the rotated values) -> (codes uint8 [n, d], scales
+    fp32 [n]) with one scale per row."""
+    r = np.asarray(rows, dtype=np.float32)
+    amax = np.abs(r).max(axis=-1) if r.shape[-1] else np.zeros(r.shape[:-1], np.float32)
+    scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    y = r / scale[..., None]                  # fp32 division, as the codes are decided
+    return e4m3_encode(y), scale
+
+
+def dequantize_fp8_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """The cache rows the codes stand for: value(code) * scale, in fp64."""
+    return e4m3_values()[np.asarray(codes)] * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+# --------------------------------------------------------------------------
 # Step 2: lightning indexer ("64 heads x 128 dims, ReLU scores weighted per
 # head") and top-k ("keeps the top 1,024 entries")
 # --------------------------------------------------------------------------

@@ -562,3 +562,52 @@ def test_csa2_full_and_reuse_layers_match_brute_force():
         ref = brute.attend(q2[t].tolist(), t, rows, sink2.tolist(), kw["scale"], kw["rope_dim"],
                            THETA)
         np.testing.assert_allclose(reuse[t], np.array(ref), atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 KV cache
+# The cache quantized after RoPE ("Partial RoPE" row of "DeepSeek-V4.1-Flash
+# vs Inkling"), read as OCP E4M3 with one fp32 scale per row: pinned to the
+# format's stated points, to torch's float8_e4m3fn conversion (a library
+# routine, round to nearest even) and to the rounding error bound.
+def test_e4m3_code_table_has_the_format_points():
+    v = oracle.e4m3_values()
+    assert v[0x7E] == 448.0 and v[0xFE] == -448.0          # largest finite
+    assert v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9   # smallest normal, subnormal
+    assert v[0x38] == 1.0 and v[0x00] == 0.0 and np.signbit(v[0x80])
+    assert [c for c in range(256) if np.isnan(v[c])] == [0x7F, 0xFF]
+    assert np.all(np.diff(v[:127]) > 0)                     # codes 0..126 increase
+    np.testing.assert_array_equal(v[128:255], -v[:127])     # sign bit
+
+
+def test_e4m3_encode_matches_torch_float8_e4m3fn():
+    rng = _rng(80)
+    v = oracle.e4m3_values()[:127]
+    mids = (v[1:] + v[:-1]) / 2                              # every tie between neighbours
+    x = np.concatenate([rng.uniform(-448, 448, 20000), rng.standard_normal(20000) * 1e-2,
+                        rng.standard_normal(5000) * 2 ** -8, mids, -mids, v, -v]).astype(np.float32)
+    ours = oracle.e4m3_encode(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_quantized_rows_round_trip_and_error_bound():
+    rng = _rng(81)
+    rows = (rng.standard_normal((40, 512)) * np.exp(rng.uniform(-6, 6, (40, 1)))).astype(np.float32)
+    rows[3] = 0.0
+    codes, scales = oracle.quantize_fp8_rows(rows)
+    back = oracle.dequantize_fp8_rows(codes, scales)
+    assert scales[3] == 1.0 and np.all(codes[3] == 0)       # an all-zero row
+    for r in range(40):
+        j = int(np.argmax(np.abs(rows[r])))
+        if rows[r, j] != 0:                                   # the largest maps to +-448
+            assert abs(oracle.e4m3_values()[codes[r, j]]) == 448.0
+    # relative half-step of 3 mantissa bits for normals, absolute half of the
+    # smallest subnormal step below 2^-6 (both in units of the row's scale)
+    y = np.abs(rows / scales[:, None].astype(np.float64))
+    bound = np.where(y >= 2.0 ** -6, y * 2.0 ** -4, 2.0 ** -10) * scales[:, None] * (1 + 1e-6)
+    assert np.all(np.abs(back - rows) <= bound)
+    # rows made of code values times a power-of-two scale come back exactly
+    exact = oracle.e4m3_values()[rng.integers(0, 127, (5, 64))] * 2.0 ** -3
+    exact[:, 0] = 448 * 2.0 ** -3
+    c2, s2 = oracle.quantize_fp8_rows(exact)
+    np.testing.assert_array_equal(oracle.dequantize_fp8_rows(c2, s2), exact)
