@@ -81,7 +81,8 @@ def _args():
                     help="csa_decode_bs32_ctx65536 (default), csa_decode_bs4_ctx1048576, "
                          "hca_decode_bs16_ctx131072, csa_prefill_T8192, "
                          "csa_decode_yarn_bs32_ctx131072, csa2_decode_bs32_ctx65536 "
-                         "(one Full + five Reuse layers) or hca_prefill_T8192")
+                         "(one Full + five Reuse layers), hca_prefill_T8192 or "
+                         "csa_decode_fp8kv_bs32_ctx65536")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--seq-len", type=int, default=0,
@@ -126,6 +127,8 @@ def _config(wl, extra=None, flush_mib=256):
     if wl.rope_factor > 1.0:
         c["rope"] = (f"theta {wl.theta:g}, YaRN factor {wl.rope_factor:g} over "
                      f"{wl.rope_orig_ctx} tokens")
+    if wl.kv_fp8:
+        c["kv_cache"] = "E4M3 codes + one fp32 scale per row, quantized after RoPE (outside the step)"
     if wl.reuse_layers:
         c["layers"] = (f"1 Full layer (indexer, top-k, attention) + {wl.reuse_layers} Reuse "
                        "layers (attention over the Full layer's entries and selection)")
@@ -164,7 +167,8 @@ def algorithmic_work(wl):
     if wl.kind == "csa_decode":
         vis = N                      # every entry is visible to the decode query
         n_rows = min(wl.topk, N) + wl.window
-        rows = n_q * n_rows * d * 2  # gathered rows (selected + window)
+        row_bytes = d + 4 if wl.kv_fp8 else d * 2   # E4M3 codes + scale, or bf16
+        rows = n_q * n_rows * row_bytes  # gathered rows (selected + window)
         pre = {}
     else:
         # causal prefill: query t sees floor((t - width) / stride) + 1 entries
@@ -319,11 +323,15 @@ def _oracle_sample(wl):
         return step, wl.n_heads, (f"one of the {wl.B} sequences per step (128-head attention "
                                   f"over its {wl.n_cmp} entries and window), fp64 NumPy oracle")
 
+    kv = {key: v(data[key][0]) for key in ("kv_cmp", "kv_raw")}
+    if wl.kv_fp8:  # the caches the quantized ones stand for (quantized outside the step)
+        kv = {key: oracle.dequantize_fp8_rows(*oracle.quantize_fp8_rows(val))
+              for key, val in kv.items()}
+
     def attend(q, idx, sink):
-        return oracle.sparse_attn(q, data["q_pos"][0], v(data["kv_cmp"][0]), idx,
-                                  v(data["kv_raw"][0]), int(data["raw_pos0"][0]),
-                                  int(data["n_raw"][0]), sink, wl.scale, wl.window,
-                                  wl.rope_dim, th)
+        return oracle.sparse_attn(q, data["q_pos"][0], kv["kv_cmp"], idx, kv["kv_raw"],
+                                  int(data["raw_pos0"][0]), int(data["n_raw"][0]), sink,
+                                  wl.scale, wl.window, wl.rope_dim, th)
 
     def step():
         qp = data["q_pos"][0]
@@ -443,6 +451,11 @@ def run_cuda(args, rank, world, local):
     if not hca:
         scores = torch.empty((Bsz, Tq, N), dtype=torch.float32, device=dev)
         idx = torch.empty((Bsz, Tq, wl.topk), dtype=torch.int32, device=dev)
+    if wl.kv_fp8:  # the caches as written: quantized after RoPE, once
+        for key in ("kv_cmp", "kv_raw"):
+            codes, scales = layer.quantize_fp8(t[key])
+            t[key + "_fp8"], t[key + "_scale"] = codes, scales
+        torch.cuda.synchronize()
     if prefill:
         t["kv_cmp"] = torch.empty((Bsz, N, wl.d), dtype=torch.bfloat16, device=dev)
         t["kv_raw"] = torch.empty((Bsz, wl.T, wl.d), dtype=torch.bfloat16, device=dev)
@@ -463,9 +476,14 @@ def run_cuda(args, rank, world, local):
             p, t["q_idx"], t["w"], t["k_idx"], t["q_pos"], t["n_cmp"], scores)))
         groups.append(("topk_select", lambda: L.csa_topk_select(
             p, scores, t["q_pos"], t["n_cmp"], idx, ws)))
-        groups.append(("sparse_attn", lambda: L.csa_sparse_attn(
-            p, t["q"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"], t["n_raw"],
-            t["sink"], out, ws)))
+        if wl.kv_fp8:
+            groups.append(("sparse_attn", lambda: L.csa_sparse_attn_fp8(
+                p, t["q"], t["q_pos"], t["kv_cmp_fp8"], t["kv_cmp_scale"], idx, t["kv_raw_fp8"],
+                t["kv_raw_scale"], t["raw_pos0"], t["n_raw"], t["sink"], out, ws)))
+        else:
+            groups.append(("sparse_attn", lambda: L.csa_sparse_attn(
+                p, t["q"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"], t["n_raw"],
+                t["sink"], out, ws)))
     R = wl.reuse_layers
     if R:
         out_r = torch.empty_like(t["q_reuse"])
@@ -582,7 +600,12 @@ def run_cuda(args, rank, world, local):
             e_start.record()
             for k in h_in:
                 d_in[k].copy_(h_in[k], non_blocking=True)
-            if wl.kind == "csa_decode":
+            if wl.kind == "csa_decode" and wl.kv_fp8:
+                _, o = layer.csa_decode_fp8(
+                    p, bf("q"), d_in["q_pos"], bf("q_idx"), d_in["w"], t["k_idx"], t["n_cmp"],
+                    t["kv_cmp_fp8"], t["kv_cmp_scale"], t["kv_raw_fp8"], t["kv_raw_scale"],
+                    t["raw_pos0"], t["n_raw"], t["sink"], lw, idx=idx, out=out)
+            elif wl.kind == "csa_decode":
                 _, o = layer.csa_decode(p, bf("q"), d_in["q_pos"], bf("q_idx"), d_in["w"],
                                         t["k_idx"], t["n_cmp"], t["kv_cmp"], t["kv_raw"],
                                         t["raw_pos0"], t["n_raw"], t["sink"], lw, idx=idx,

@@ -245,6 +245,42 @@ csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const void* q,
                       const int32_t* n_raw, int32_t raw_max, const float* sink, int32_t B,
                       int32_t Tq, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* KV cache quantized after RoPE ("DeepSeek-V4.1-Flash vs Inkling", "Partial
+ * RoPE" row: the KV cache is quantized after RoPE; the pages give no
+ * format).  Format of this library: OCP 8-bit float E4M3 codes (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits, no infinities, largest finite
+ * 448) with one fp32 scale per cache row.
+ *   rows   [n][d] (dtype bf16 or fp32) rotated cache rows, d a multiple of 32
+ *          in [32, 1024]
+ *   codes  [n][d] uint8: code = x / scale rounded to the nearest E4M3 value
+ *          (ties to even), saturated at +-448
+ *   scales [n] fp32: scale = max|row| / 448, 1 for an all-zero row
+ * The scale and the division are IEEE fp32 (correctly rounded). */
+csa_status_t csa_quantize_fp8(csa_dtype_t dtype, const void* rows, int64_t n, int32_t d,
+                              uint8_t* codes, float* scales, void* stream);
+
+/* Steps 3/4 over FP8 caches: csa_sparse_attn and hca_attn with kv_cmp
+ * [B][n_max][d] and kv_raw [B][raw_max][d] holding E4M3 codes and
+ * cmp_scale [B][n_max], raw_scale [B][raw_max] their row scales (as
+ * csa_quantize_fp8 writes them).  A row stands for code value x scale; the
+ * kernel rounds that product to bf16 once before the products.  q and out
+ * are bf16; the tensor-core shape only (d = 512, 128 heads, rope_dim <= 128,
+ * topk (or n_max) + window + 8 <= 2048 rows), CSA_ERR_UNSUPPORTED_SHAPE
+ * otherwise.  ws: csa_workspace_size(CSA_OP_SPARSE_ATTN / CSA_OP_HCA_ATTN). */
+csa_status_t csa_sparse_attn_fp8(const csa_params_t* p, const void* q, const int32_t* q_pos,
+                                 const uint8_t* kv_cmp, const float* cmp_scale,
+                                 const int32_t* idx, int32_t n_max, const uint8_t* kv_raw,
+                                 const float* raw_scale, const int32_t* raw_pos0,
+                                 const int32_t* n_raw, int32_t raw_max, const float* sink,
+                                 int32_t B, int32_t Tq, void* out, void* ws, size_t ws_bytes,
+                                 void* stream);
+csa_status_t hca_attn_fp8(const csa_params_t* p, const void* q, const int32_t* q_pos,
+                          const uint8_t* kv_cmp, const float* cmp_scale, const int32_t* n_cmp,
+                          int32_t n_max, const uint8_t* kv_raw, const float* raw_scale,
+                          const int32_t* raw_pos0, const int32_t* n_raw, int32_t raw_max,
+                          const float* sink, int32_t B, int32_t Tq, void* out, void* ws,
+                          size_t ws_bytes, void* stream);
+
 /* Indexer + top-k that allocates nothing: the same computation and
  * arguments as csa_index_topk, without `ws`.  The pages have no counterpart
  * of this call; it serves callers that cannot call cudaMalloc or hand out a

@@ -102,6 +102,10 @@ def _load():
     lib.csa_sparse_attn.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P,
                                     _I, _I, _P, _P, ctypes.c_size_t, _P]
     lib.hca_attn.argtypes = list(lib.csa_sparse_attn.argtypes)
+    lib.csa_quantize_fp8.argtypes = [ctypes.c_int, _P, ctypes.c_int64, _I, _P, _P, _P]
+    lib.csa_sparse_attn_fp8.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _P, _I,
+                                        _I, _P, _P, ctypes.c_size_t, _P]
+    lib.hca_attn_fp8.argtypes = list(lib.csa_sparse_attn_fp8.argtypes)
     lib.csa_index_topk_noalloc.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _P, _I, _I, _I, _P,
                                            _P]
     lib.csa_poll_device_error.argtypes = [_P]
@@ -113,7 +117,7 @@ def _load():
     lib.csa_last_device_error_site.argtypes = []
     for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
               "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error",
-              "csa_compress_append",
+              "csa_compress_append", "csa_quantize_fp8", "csa_sparse_attn_fp8", "hca_attn_fp8",
               "csa_index_topk_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -321,3 +325,57 @@ def csa_poll_device_error(stream=None):
 def csa_last_device_error_site() -> int:
     """Kernel source line of the check behind the last device error polled."""
     return int(_load().csa_last_device_error_site())
+
+
+def csa_quantize_fp8(rows, codes, scales, stream=None):
+    """Cache rows [..., d] (bf16 or fp32, already rotated) -> E4M3 codes
+    [..., d] uint8 and one fp32 scale per row [...]."""
+    import torch
+    _req(rows, "rows")
+    _req(codes, "codes", torch.uint8, rows.dim())
+    _req(scales, "scales", torch.float32, rows.dim() - 1)
+    d = rows.shape[-1]
+    n = rows.numel() // d if d else 0
+    if tuple(codes.shape) != tuple(rows.shape) or tuple(scales.shape) != tuple(rows.shape[:-1]):
+        raise ValueError("codes must match rows and scales its leading dims")
+    _check(_load().csa_quantize_fp8(_dtype_code(rows), _ptr(rows), n, d, _ptr(codes), _ptr(scales),
+                                    _stream(stream)))
+
+
+def _attn_fp8(fn, p, q, q_pos, kv_cmp, cmp_scale, sel, kv_raw, raw_scale, raw_pos0, n_raw, sink,
+              out, ws, stream):
+    import torch
+    _req(q, "q", torch.bfloat16, 4)
+    _req(q_pos, "q_pos", torch.int32, 2)
+    _req(kv_cmp, "kv_cmp", torch.uint8, 3)
+    _req(cmp_scale, "cmp_scale", torch.float32, 2)
+    _req(kv_raw, "kv_raw", torch.uint8, 3)
+    _req(raw_scale, "raw_scale", torch.float32, 2)
+    _req(raw_pos0, "raw_pos0", torch.int32, 1)
+    _req(n_raw, "n_raw", torch.int32, 1)
+    _req(sink, "sink", torch.float32, 1)
+    _req(out, "out", torch.bfloat16, 4)
+    B, Tq = q_pos.shape
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(fn(ctypes.byref(p.c()), _ptr(q), _ptr(q_pos), _ptr(kv_cmp), _ptr(cmp_scale), _ptr(sel),
+              kv_cmp.shape[1], _ptr(kv_raw), _ptr(raw_scale), _ptr(raw_pos0), _ptr(n_raw),
+              kv_raw.shape[1], _ptr(sink), B, Tq, _ptr(out), _ptr(ws), nb, _stream(stream)))
+
+
+def csa_sparse_attn_fp8(p: Params, q, q_pos, kv_cmp, cmp_scale, idx, kv_raw, raw_scale, raw_pos0,
+                        n_raw, sink, out, ws=None, stream=None):
+    """As csa_sparse_attn over FP8 caches: kv_cmp [B][n_max][d] and kv_raw
+    [B][raw_max][d] E4M3 codes with row scales [B][n_max], [B][raw_max]."""
+    import torch
+    _req(idx, "idx", torch.int32, 3)
+    _attn_fp8(_load().csa_sparse_attn_fp8, p, q, q_pos, kv_cmp, cmp_scale, idx, kv_raw, raw_scale,
+              raw_pos0, n_raw, sink, out, ws, stream)
+
+
+def hca_attn_fp8(p: Params, q, q_pos, kv_cmp, cmp_scale, n_cmp, kv_raw, raw_scale, raw_pos0,
+                 n_raw, sink, out, ws=None, stream=None):
+    """As hca_attn over FP8 caches (codes and row scales)."""
+    import torch
+    _req(n_cmp, "n_cmp", torch.int32, 1)
+    _attn_fp8(_load().hca_attn_fp8, p, q, q_pos, kv_cmp, cmp_scale, n_cmp, kv_raw, raw_scale,
+              raw_pos0, n_raw, sink, out, ws, stream)

@@ -48,12 +48,20 @@
 // O and its (m, l) to the workspace through shared memory and bulk copies;
 // k_attn_merge, launched right after, combines the splits.
 //
+// FP8 KV cache (kFp8): the caches hold E4M3 codes with one fp32 scale per
+// row (quantized after RoPE).  Two gather warps land each chunk's codes (64
+// rows x 128 B) in the upper half of its ring slot and its row scales in
+// shared memory; two expanding warps rewrite each row in place as bf16
+// (code value x row scale, rounded once) in the slot's 128B-swizzled layout
+// and release the slot to the MMA.  The rest of the kernel is the bf16 one.
+//
 // Every mbarrier wait is bounded (a.wait_ns); a wait that runs out records
 // CSA_ERR_DEVICE_TIMEOUT and the CTA winds down: it drains every copy and
 // MMA it issued and every partner store it expects, reaches every cluster
 // barrier, frees TMEM and exits.
 #pragma once
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -76,7 +84,8 @@ constexpr int kApMaxSplits = 8;                      // split-KV parts per query
 constexpr int kApSlabBytes = kApHeads * 32 * 2;      // 32 dims of fp16 O, 128 heads
 constexpr int kApOutBoxBytes = kApHeads * 64;        // 32 dims of bf16 output, 128 heads
 constexpr int kApSlabs = kApHalf / 32;
-constexpr int kApThreads = 288;  // 9 warps
+constexpr int kApThreads = 288;      // 9 warps
+constexpr int kApThreadsFp8 = 352;   // FP8 caches: 2 more expanding warps (9, 10)
 constexpr float kApRescaleLog2 = 8.0f;
 constexpr int kApXOff = kApSlots * kApChunkBytes;
 constexpr int kApMiscOff = kApXOff + kApXBufs * kApXBytes;
@@ -90,6 +99,8 @@ struct AttnPairArgs {
   const int* n_cmp;  // HCA
   int n_max;
   const __nv_bfloat16* kv_raw;
+  const float* cmp_scale;  // FP8 caches: [B * n_max] and [B * raw_max] row scales
+  const float* raw_scale;
   const int* raw_pos0;
   const int* n_raw;
   int raw_max;
@@ -108,6 +119,8 @@ struct ApMisc {
   int rows[kApRowCap];  // gather row coordinates
   float cs[kApMaxRope / 2], sn[kApMaxRope / 2];
   uint64_t full[kApSlots], empty[kApSlots];
+  uint64_t stage[kApSlots];  // FP8: a chunk's codes have landed in its slot
+  float scl[kApSlots][kApTile];  // FP8: the row scales of each slot's chunk
   uint64_t s_full[2], p_full[2], pv_done[2], xfull[kApXBufs];
   uint64_t q_tma, q_ready, rows_ready, rope_ready, mma_drain;
   uint32_t tmem_base;
@@ -162,6 +175,47 @@ __device__ __forceinline__ uint32_t ap_swz64(int r, int u) {
   return (uint32_t)(r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
 }
 
+// FP8 caches: expand row r of a chunk from its E4M3 codes (128 B at the
+// upper half of the slot, row-major) to bf16 (code value x scale, rounded
+// once): dims 0-63 into the lower half, 64-127 into the upper half over the
+// row's own codes, both in the 128B-swizzled layout the MMA reads.  The
+// thread loads all of the row's codes before it writes any byte.
+__device__ __forceinline__ void ap_expand_fp8_row(uint8_t* slot, int r, float scale) {
+  const uint4* src = reinterpret_cast<const uint4*>(slot + kApChunkBytes / 2 + r * 128);
+  uint4 c[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) c[u] = src[u];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {  // codes 16u .. 16u + 15
+    const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int hw = 0; hw < 2; ++hw) {  // codes 4k + 2hw, 4k + 2hw + 1
+        const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(
+            (__nv_fp8x2_storage_t)((w[k] >> (16 * hw)) & 0xFFFFu), __NV_E4M3);
+        const float2 f = __half22float2(__half2(h2));
+        o[2 * k + hw] = ap_bf16x2(f.x * scale, f.y * scale);
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {  // bf16 unit 2u + v of the row (8 dims)
+      const int unit = 2 * u + v, hh = unit >> 3, uu = unit & 7;
+      *reinterpret_cast<uint4*>(slot + hh * (kApChunkBytes / 2) + r * 128 + ((uu ^ (r & 7)) << 4)) =
+          make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+    }
+  }
+}
+
+// Zero row r of a chunk (both halves): masked rows past the split's end.
+__device__ __forceinline__ void ap_zero_row(uint8_t* slot, int r) {
+#pragma unroll
+  for (int unit = 0; unit < 16; ++unit)
+    *reinterpret_cast<uint4*>(slot + (unit >> 3) * (kApChunkBytes / 2) + r * 128 +
+                              ((unit & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // All 128 threads of warps 0-3 agree on `ok` (named barrier 1).
 __device__ __forceinline__ bool ap_softmax_all(bool ok) {
   uint32_t all;
@@ -174,8 +228,8 @@ __device__ __forceinline__ bool ap_softmax_all(bool ok) {
   return all != 0;
 }
 
-template <bool kHca>
-__global__ void __launch_bounds__(kApThreads, 1)
+template <bool kHca, bool kFp8>
+__global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
     k_attn_pair(AttnPairArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_out,
                 const __grid_constant__ CUtensorMap tm_cmp,
@@ -203,8 +257,9 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kApSlots; ++s) {
-      mbar_init(&sm.full[s], 1);  // the producer warp's expect_tx + the chunk's bytes
+      mbar_init(&sm.full[s], kFp8 ? 2 : 1);  // expect_tx + the chunk's bytes (FP8: 2 expanders)
       mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.stage[s], 1);  // FP8: expect_tx + the codes' bytes
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
@@ -657,6 +712,74 @@ __global__ void __launch_bounds__(kApThreads, 1)
         }
       }
     }
+  } else if (kFp8 && warp != 8) {
+    // ======================= FP8 caches: warps 4-5 gather, 6, 7, 9, 10 expand
+    // Chunk n = 2i + c of tile i goes to ring slot n % kApSlots.  Warp 4 + c
+    // gathers chunk c of every tile: lanes 0-15 each the codes of rows
+    // 4l .. 4l + 3 (128 dims, 128 B a row) into the upper half of the slot,
+    // and the rows' scales into sm.scl.  Expanding warp e (warps 6, 7, 9,
+    // 10 are e = 0..3) takes chunk c = e % 2, rows 32 (e / 2) + lane: waits
+    // for the codes, expands its rows to bf16 in place, and arrives on the
+    // slot's full barrier (two arrivals release it to the MMA).  The gathers
+    // run ahead of the expansion by up to the ring.
+    load_split();
+    const int ex = warp < 8 ? warp - 6 : warp - 7;  // expander index (warps 6, 7, 9, 10)
+    const int ck = warp < 6 ? warp - 4 : ex & 1;
+    const int ps = (sm.n_sel + 3) & ~3;
+    bool okp = __all_sync(0xffffffffu, rows_ok);
+    if (warp < 6) {
+      bool staged = false;  // q staging slots handed back
+      for (int i = 0; i < ntile && okp; ++i) {
+        const int n = 2 * i + ck;
+        const int slot = n % kApSlots;
+        if (lane == 0) {
+          okp = mbar_wait(&sm.empty[slot], ((uint32_t)(n / kApSlots) & 1u) ^ 1u, abortp, wait_ns);
+          if (okp && !staged && slot >= kApQSlot0) {  // slot still holds q staging
+            okp = mbar_wait(&sm.q_ready, 0, abortp, wait_ns);
+            staged = true;
+          }
+        }
+        okp = __shfl_sync(0xffffffffu, okp ? 1 : 0, 0) != 0;
+        if (!okp) break;
+        const int g0 = r_lo + i * kApTile;  // list index of the chunk's row 0
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int gi = g0 + lane + 32 * q;
+          sm.scl[slot][lane + 32 * q] =
+              gi < r_hi ? (gi < ps ? a.cmp_scale : a.raw_scale)[sm.rows[gi]] : 0.f;
+        }
+        const int g = g0 + 4 * lane;
+        const bool gv = lane < 16 && g < r_hi;
+        const unsigned vmask = __ballot_sync(0xffffffffu, gv);  // also orders the scales
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sm.stage[slot], (uint32_t)__popc(vmask) * 512u);
+          sm.last_n[slot] = n;
+        }
+        __syncwarp();
+        if (gv)
+          tma_gather4(ring + slot * kApChunkBytes + kApChunkBytes / 2 + lane * 512,
+                      g < ps ? &tm_cmp : &tm_raw, &sm.stage[slot], dim0 + ck * 128, sm.rows[g],
+                      sm.rows[g + 1], sm.rows[g + 2], sm.rows[g + 3]);
+      }
+    } else {
+      for (int i = 0; i < ntile && okp; ++i) {
+        const int n = 2 * i + ck;
+        const int slot = n % kApSlots;
+        okp = __all_sync(0xffffffffu, mbar_wait(&sm.stage[slot], (uint32_t)(n / kApSlots) & 1u,
+                                                abortp, wait_ns));
+        if (!okp) break;
+        const int g0 = r_lo + i * kApTile;
+        uint8_t* sl = ring + slot * kApChunkBytes;
+        const int r = 32 * (ex >> 1) + lane;
+        if (g0 + r < r_hi)
+          ap_expand_fp8_row(sl, r, sm.scl[slot][r]);
+        else
+          ap_zero_row(sl, r);
+        fence_proxy_async_shared();  // read by the MMA (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.full[slot]);
+      }
+    }
   } else if (warp < 8) {
     // ======================= gather producers (warps 4-7)
     // Chunk n (tile n / 2, dims dim0 + 128 (n % 2)) goes to ring slot
@@ -807,7 +930,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
     mbar_drain(&sm.q_tma, 0, kApDrainNs);
     for (int s = 0; s < kApSlots; ++s) {
       const int n = sm.last_n[s];
-      if (n >= 0) mbar_drain(&sm.full[s], (uint32_t)(n / kApSlots) & 1u, kApDrainNs);
+      if (n >= 0)
+        mbar_drain(kFp8 ? &sm.stage[s] : &sm.full[s], (uint32_t)(n / kApSlots) & 1u, kApDrainNs);
     }
   }
   tc_fence_before();

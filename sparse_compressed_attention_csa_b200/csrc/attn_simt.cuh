@@ -28,6 +28,8 @@ struct AttnArgs {
   const int* n_raw;
   int raw_max;
   const float* sink;
+  const float* cmp_scale;  // FP8 caches (tensor-core path only): row scales
+  const float* raw_scale;
   int B, Tq, H, d, rope_dim, topk, window, width, stride;
   float scale;  // with the extended RoPE's temperature
   RopeSpec rope;

@@ -16,6 +16,7 @@
 #include "attn_simt.cuh"
 #include "common.cuh"
 #include "compress.cuh"
+#include "quantize.cuh"
 #include "csa.h"
 #include "indexer_simt.cuh"
 #include "indexer_tc.cuh"
@@ -264,6 +265,22 @@ csa_status_t make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, ui
   return CSA_OK;
 }
 
+// Row-gather map over E4M3 codes [rows][inner] (bytes), no swizzle.
+csa_status_t make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                          uint32_t box_inner) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return CSA_OK;
+}
+
 size_t scores_bytes(int B, int Tq, int n_max) {
   return round_up((size_t)B * Tq * (size_t)n_max * sizeof(float), 256);
 }
@@ -324,8 +341,9 @@ TopkPlan topk_plan(const csa_params_t* p, int B, int Tq, int n_max) {
     const int c = (n_max + kTopkMid - 1) / kTopkMid;
     if (rows * c <= num_sms()) return {1, kTopkMid, 0, c};
   }
-  // few very long rows: a cluster of up to 16 CTAs of 16,384 entries per row
-  if (n_max > kTopkMaxCluster * kTopkMid && n_max <= kTopkMaxWideCluster * kTopkBig) {
+  // few long rows (or too many rows for clusters of 4,096-entry CTAs): a
+  // cluster of up to 16 CTAs of 16,384 entries per row
+  if (n_max > kTopkBig && n_max <= kTopkMaxWideCluster * kTopkBig) {
     const int c = (n_max + kTopkBig - 1) / kTopkBig;
     if (rows * c <= num_sms() && wide_topk_cluster_fits(c)) return {1, kTopkBig, 0, c};
   }
@@ -767,7 +785,7 @@ static csa_status_t launch_attn_simt(const AttnArgs& a, csa_dtype_t dtype, cudaS
   return launched("k_attn_simt");
 }
 
-template <bool kHca>
+template <bool kHca, bool kFp8 = false>
 static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, void* ws,
                                    size_t ws_bytes, cudaStream_t s) {
   const int sp = attn_splits(p, kHca, g.B, g.Tq, g.n_max);
@@ -783,6 +801,8 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   a.n_cmp = g.n_cmp;
   a.n_max = g.n_max;
   a.kv_raw = (const __nv_bfloat16*)g.kv_raw;
+  a.cmp_scale = g.cmp_scale;
+  a.raw_scale = g.raw_scale;
   a.raw_pos0 = g.raw_pos0;
   a.n_raw = g.n_raw;
   a.raw_max = g.raw_max;
@@ -815,14 +835,22 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   // read, and its map is made over q instead
   const uint64_t n_cmp_rows = (uint64_t)g.B * g.n_max, n_raw_rows = (uint64_t)g.B * g.raw_max;
   const uint64_t n_q_rows = (uint64_t)g.B * g.Tq * kApHeads;
-  CSA_CHECK(make_tmap_bf16(&tc, n_cmp_rows ? g.kv_cmp : g.q, kApDim,
-                           n_cmp_rows ? n_cmp_rows : n_q_rows, 64, 1));
-  CSA_CHECK(make_tmap_bf16(&tr, n_raw_rows ? g.kv_raw : g.q, kApDim,
-                           n_raw_rows ? n_raw_rows : n_q_rows, 64, 1));
-  CSA_CHECK(set_smem_attr(k_attn_pair<kHca>, kApSmemBytes, "k_attn_pair"));
+  if (kFp8) {  // E4M3 codes: one-row boxes of 128 dims (128 B)
+    CSA_CHECK(make_tmap_u8(&tc, n_cmp_rows ? g.kv_cmp : g.q, kApDim,
+                           n_cmp_rows ? n_cmp_rows : n_q_rows, 128));
+    CSA_CHECK(make_tmap_u8(&tr, n_raw_rows ? g.kv_raw : g.q, kApDim,
+                           n_raw_rows ? n_raw_rows : n_q_rows, 128));
+  } else {
+    CSA_CHECK(make_tmap_bf16(&tc, n_cmp_rows ? g.kv_cmp : g.q, kApDim,
+                             n_cmp_rows ? n_cmp_rows : n_q_rows, 64, 1));
+    CSA_CHECK(make_tmap_bf16(&tr, n_raw_rows ? g.kv_raw : g.q, kApDim,
+                             n_raw_rows ? n_raw_rows : n_q_rows, 64, 1));
+  }
+  CSA_CHECK(set_smem_attr(k_attn_pair<kHca, kFp8>, kApSmemBytes, "k_attn_pair"));
   dim3 grid((unsigned)(2 * sp), (unsigned)(g.B * g.Tq));
-  cudaError_t e =
-      launch_ex(k_attn_pair<kHca>, grid, dim3(kApThreads), kApSmemBytes, s, 2, a, tq, to, tc, tr);
+  cudaError_t e = launch_ex(k_attn_pair<kHca, kFp8>, grid,
+                            dim3(kFp8 ? kApThreadsFp8 : kApThreads), kApSmemBytes, s, 2, a, tq, to,
+                            tc, tr);
   if (e != cudaSuccess) return cuda_fail(e, "k_attn_pair");
   CSA_CHECK(launched("k_attn_pair"));
   if (sp == 1) return CSA_OK;
@@ -849,6 +877,7 @@ static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32
   AttnArgs a;
   a.q = q; a.q_pos = q_pos; a.kv_cmp = kv_cmp; a.idx = idx; a.n_cmp = n_cmp; a.n_max = n_max;
   a.kv_raw = kv_raw; a.raw_pos0 = raw_pos0; a.n_raw = n_raw; a.raw_max = raw_max; a.sink = sink;
+  a.cmp_scale = nullptr; a.raw_scale = nullptr;
   a.B = B; a.Tq = Tq; a.H = p->n_heads; a.d = p->d; a.rope_dim = p->rope_dim; a.topk = p->topk;
   a.window = p->window; a.width = p->width; a.stride = p->stride; a.scale = attn_scale(p);
   a.rope = rope_spec(p); a.out = out;
@@ -887,6 +916,88 @@ CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const vo
   if (attn_tc_ok(p, dtype, true, n_max))
     return launch_attn_tc<true>(p, a, ws, ws_bytes, (cudaStream_t)stream);
   return launch_attn_simt<true>(a, dtype, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------
+// FP8 KV cache (quantized after RoPE): quantizer and the attention calls
+// over E4M3 caches.
+// ---------------------------------------------------------------------------
+CSA_API csa_status_t csa_quantize_fp8(csa_dtype_t dtype, const void* rows, int64_t n, int32_t d,
+                                      uint8_t* codes, float* scales, void* stream) {
+  CSA_CHECK(check_dtype(dtype));
+  if (n < 0 || d < 8 || d > 1024 || (d & 31))
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "n=%lld d=%d: d a multiple of 32 in [32, 1024]",
+                (long long)n, d);
+  if (n == 0) return CSA_OK;
+  CSA_CHECK(check_ptr(rows, "rows"));
+  CSA_CHECK(check_ptr(codes, "codes"));
+  CSA_CHECK(check_ptr(scales, "scales"));
+  CSA_CHECK(check_device());
+  const long long ctas = (n + kQuantWarps - 1) / kQuantWarps;
+  if (ctas > 2147483647LL) return fail(CSA_ERR_UNSUPPORTED_SHAPE, "n=%lld", (long long)n);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == CSA_BF16)
+    k_quantize_fp8<__nv_bfloat16><<<(unsigned)ctas, 32 * kQuantWarps, 0, s>>>(
+        (const __nv_bfloat16*)rows, n, d, codes, scales);
+  else
+    k_quantize_fp8<float><<<(unsigned)ctas, 32 * kQuantWarps, 0, s>>>((const float*)rows, n, d,
+                                                                      codes, scales);
+  return launched("k_quantize_fp8");
+}
+
+static csa_status_t attn_fp8_checks(const csa_params_t* p, bool hca, const void* q,
+                                    const int32_t* q_pos, const void* kv_cmp,
+                                    const float* cmp_scale, int32_t n_max, const void* kv_raw,
+                                    const float* raw_scale, const int32_t* raw_pos0,
+                                    const int32_t* n_raw, int32_t raw_max, const float* sink,
+                                    int32_t B, int32_t Tq, void* out) {
+  CSA_CHECK(attn_common_checks(p, CSA_BF16, q, q_pos, kv_cmp, n_max, kv_raw, raw_pos0, n_raw,
+                               raw_max, sink, B, Tq, out));
+  CSA_CHECK(check_ptr(cmp_scale, "cmp_scale", n_max == 0));
+  CSA_CHECK(check_ptr(raw_scale, "raw_scale", raw_max == 0));
+  if (!attn_tc_ok(p, CSA_BF16, hca, n_max))
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE,
+                "FP8 caches take the tensor-core path only: d = 512, 128 heads, rope_dim <= %d, "
+                "at most %d rows per query", kApMaxRope, kApRowCap - 8);
+  return CSA_OK;
+}
+
+CSA_API csa_status_t csa_sparse_attn_fp8(const csa_params_t* p, const void* q,
+                                         const int32_t* q_pos, const uint8_t* kv_cmp,
+                                         const float* cmp_scale, const int32_t* idx,
+                                         int32_t n_max, const uint8_t* kv_raw,
+                                         const float* raw_scale, const int32_t* raw_pos0,
+                                         const int32_t* n_raw, int32_t raw_max, const float* sink,
+                                         int32_t B, int32_t Tq, void* out, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  CSA_CHECK(attn_fp8_checks(p, false, q, q_pos, kv_cmp, cmp_scale, n_max, kv_raw, raw_scale,
+                            raw_pos0, n_raw, raw_max, sink, B, Tq, out));
+  CSA_CHECK(check_topk(p));
+  CSA_CHECK(check_ptr(idx, "idx"));
+  CSA_CHECK(check_device());
+  AttnArgs a = make_attn_args(p, q, q_pos, kv_cmp, idx, nullptr, n_max, kv_raw, raw_pos0, n_raw,
+                              raw_max, sink, B, Tq, out);
+  a.cmp_scale = cmp_scale;
+  a.raw_scale = raw_scale;
+  return launch_attn_tc<false, true>(p, a, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+CSA_API csa_status_t hca_attn_fp8(const csa_params_t* p, const void* q, const int32_t* q_pos,
+                                  const uint8_t* kv_cmp, const float* cmp_scale,
+                                  const int32_t* n_cmp, int32_t n_max, const uint8_t* kv_raw,
+                                  const float* raw_scale, const int32_t* raw_pos0,
+                                  const int32_t* n_raw, int32_t raw_max, const float* sink,
+                                  int32_t B, int32_t Tq, void* out, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  CSA_CHECK(attn_fp8_checks(p, true, q, q_pos, kv_cmp, cmp_scale, n_max, kv_raw, raw_scale,
+                            raw_pos0, n_raw, raw_max, sink, B, Tq, out));
+  CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
+  CSA_CHECK(check_device());
+  AttnArgs a = make_attn_args(p, q, q_pos, kv_cmp, nullptr, n_cmp, n_max, kv_raw, raw_pos0,
+                              n_raw, raw_max, sink, B, Tq, out);
+  a.cmp_scale = cmp_scale;
+  a.raw_scale = raw_scale;
+  return launch_attn_tc<true, true>(p, a, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -7,6 +7,7 @@ call the C ABI.  Every step runs in the CUDA library.
     HCA prefill: hca_prefill(p, x, gate, q, sink) -> (kv_cmp, kv_raw, out)
     CSA2 reuse layer: reuse_attn(p, q, ..., kv_cmp, idx, ...) -> out
     decode-time append: append_tokens(p, x, gate, x_pos0, t_old, t_new, ...)
+    FP8 caches: quantize_fp8(rows) -> (codes, scales); csa_decode_fp8(...)
 """
 from __future__ import annotations
 
@@ -122,3 +123,31 @@ def append_tokens(p: L.Params, x, gate, x_pos0, t_old, t_new, max_new: int, kv_c
     token x_pos0[b] + i at row i."""
     L.csa_compress_append(p, x, gate, x_pos0, t_old, t_new, max_new, kv_cmp, kv_raw, raw_pos0,
                           stream)
+
+
+def quantize_fp8(rows, stream=None):
+    """Cache rows [..., d] (rotated) -> (E4M3 codes uint8 [..., d], fp32
+    scales [...]), one scale per row: the KV cache quantized after RoPE."""
+    codes = torch.empty(rows.shape, dtype=torch.uint8, device=rows.device)
+    scales = torch.empty(rows.shape[:-1], dtype=torch.float32, device=rows.device)
+    L.csa_quantize_fp8(rows, codes, scales, stream)
+    return codes, scales
+
+
+def csa_decode_fp8(p: L.Params, q, q_pos, q_idx, w, k_idx, n_cmp, kv_cmp, cmp_scale, kv_raw,
+                   raw_scale, raw_pos0, n_raw, sink, ws: Workspace | None = None, idx=None,
+                   out=None, stream=None):
+    """csa_decode over FP8 caches (codes and row scales from quantize_fp8)."""
+    ws = ws or Workspace(q.device)
+    B, Tq = q_pos.shape
+    n_max = k_idx.shape[1]
+    if idx is None:
+        idx = torch.empty((B, Tq, p.topk), dtype=torch.int32, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    nb = L.csa_workspace_size(p, L.CSA_OP_INDEX_TOPK, B, Tq, n_max)
+    L.csa_index_topk(p, q_idx, w, k_idx, q_pos, n_cmp, idx, ws.get(nb), stream)
+    nb = L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, B, Tq, kv_cmp.shape[1])
+    L.csa_sparse_attn_fp8(p, q, q_pos, kv_cmp, cmp_scale, idx, kv_raw, raw_scale, raw_pos0, n_raw,
+                          sink, out, ws.get(nb), stream)
+    return idx, out

@@ -69,6 +69,7 @@ class Workload:
     rope_beta_fast: float = 32.0
     rope_beta_slow: float = 1.0
     reuse_layers: int = 0        # layers attending over this layer's entries and selection
+    kv_fp8: bool = False         # attention over the caches quantized to E4M3 after RoPE
 
     @property
     def scale(self) -> float:
@@ -121,6 +122,14 @@ CSA2_DECODE = Workload(
     width=2, stride=2, topk=512, theta=160000.0, rope_factor=16.0, rope_orig_ctx=65536,
     reuse_layers=5)
 
+# The 64K-context decode batch over the KV cache quantized after RoPE
+# ("DeepSeek-V4.1-Flash vs Inkling", "Partial RoPE" row), here E4M3 codes
+# with one fp32 scale per row: the same inputs, the caches quantized once
+# when written (outside the step).
+CSA_DECODE_FP8 = Workload(
+    name="csa_decode_fp8kv_bs32_ctx65536", kind="csa_decode", dtype="bf16", B=32, T=65536,
+    seed=2, kv_fp8=True)
+
 # HCA on a prefill sequence ("Heavily Compressed Attention" row: 128 tokens
 # -> 1 entry, dense attention over every entry plus the window), the CSA
 # prefill's length: 64 entries, every token a causal query.
@@ -130,7 +139,7 @@ HCA_PREFILL_8K = Workload(
 
 WORKLOADS = {w.name: w for w in (TINY_F32, CSA_DECODE_64K, CSA_PREFILL_8K, CSA_DECODE_1M,
                                  HCA_DECODE_128K, CSA_DECODE_YARN, CSA2_DECODE,
-                                 HCA_PREFILL_8K)}
+                                 HCA_PREFILL_8K, CSA_DECODE_FP8)}
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:

@@ -327,6 +327,7 @@ def _adversarial_rows(rng, n):
     (20000, 1024, 3, 700),     # cluster of 5, fewer visible than k
     (5000, 1024, 84, None),    # one 16384-entry block per row
     (1500, 64, 20, None),      # one 2048-entry block per row
+    (32767, 1024, 32, None),   # 32 rows x 8 CTAs of 4096 do not fit: cluster of 2 of 16384
     (40000, 1024, 7, None),    # cluster of 3 CTAs of 16384 entries
     (70000, 3000, 3, None),    # cluster of 5 of 16384, k = 3000
     (262143, 1024, 4, None),   # cluster of 16 of 16384 (the 1M-context rows)
