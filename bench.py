@@ -446,8 +446,10 @@ def run_cuda(args, rank, world, local):
     hca = wl.kind in ("hca_decode", "hca_prefill")
     prefill = wl.kind in ("csa_prefill", "hca_prefill")
     ops = [L.CSA_OP_HCA_ATTN] if hca else [L.CSA_OP_TOPK_SELECT, L.CSA_OP_SPARSE_ATTN]
-    ws = torch.empty(max([L.csa_workspace_size(p, o, Bsz, Tq, N) for o in ops] + [256]),
-                     dtype=torch.uint8, device=dev)
+    ws_sizes = [L.csa_workspace_size(p, o, Bsz, Tq, N) for o in ops]
+    if wl.reuse_layers:  # all Reuse layers in one call: layers x B query rows
+        ws_sizes.append(L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, wl.reuse_layers * Bsz, Tq, N))
+    ws = torch.empty(max(ws_sizes + [256]), dtype=torch.uint8, device=dev)
     if not hca:
         scores = torch.empty((Bsz, Tq, N), dtype=torch.float32, device=dev)
         idx = torch.empty((Bsz, Tq, wl.topk), dtype=torch.int32, device=dev)
@@ -488,11 +490,9 @@ def run_cuda(args, rank, world, local):
     if R:
         out_r = torch.empty_like(t["q_reuse"])
 
-        def reuse_layers():
-            for r in range(R):
-                L.csa_sparse_attn(p, t["q_reuse"][r], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"],
-                                  t["raw_pos0"], t["n_raw"], t["sink_reuse"][r], out_r[r], ws)
-        groups.append(("reuse_attn", reuse_layers))
+        groups.append(("reuse_attn", lambda: L.csa_reuse_attn(
+            p, t["q_reuse"], t["q_pos"], t["kv_cmp"], idx, t["kv_raw"], t["raw_pos0"],
+            t["n_raw"], t["sink_reuse"], out_r, ws)))
 
     mib = max(args.flush_mib, 0)
     flush = torch.empty(mib << 20, dtype=torch.uint8, device=dev)
@@ -610,11 +610,10 @@ def run_cuda(args, rank, world, local):
                                         t["k_idx"], t["n_cmp"], t["kv_cmp"], t["kv_raw"],
                                         t["raw_pos0"], t["n_raw"], t["sink"], lw, idx=idx,
                                         out=out)
-                for r in range(R):
-                    layer.reuse_attn(p, bf("q_reuse")[r], d_in["q_pos"], t["kv_cmp"], idx,
-                                     t["kv_raw"], t["raw_pos0"], t["n_raw"], t["sink_reuse"][r],
-                                     lw, out=out_r[r])
                 if R:
+                    layer.reuse_attn(p, bf("q_reuse"), d_in["q_pos"], t["kv_cmp"], idx,
+                                     t["kv_raw"], t["raw_pos0"], t["n_raw"], t["sink_reuse"], lw,
+                                     out=out_r)
                     h_out_r.copy_(out_r.view(torch.int16), non_blocking=True)
             elif wl.kind == "hca_decode":
                 o = layer.hca_decode(p, bf("q"), d_in["q_pos"], t["kv_cmp"], t["n_cmp"],

@@ -235,6 +235,22 @@ csa_status_t csa_sparse_attn(const csa_params_t* p, csa_dtype_t dtype, const voi
                              int32_t B, int32_t Tq, void* out, void* ws, size_t ws_bytes,
                              void* stream);
 
+/* CSA2 Reuse layers ("DeepSeek-V4.1-Flash vs Inkling", row "CSA2 encoder
+ * layers (2x compression, Full + Reuse)": the KV is computed in 3 of 18
+ * layers, the rest reuse that KV and its top-512 selection): csa_sparse_attn
+ * for `layers` layers at once, each with its own queries, sink and output,
+ * all over the same entries, selection and window.
+ *   q    [layers][B][Tq][H][d], sink [layers][H], out [layers][B][Tq][H][d]
+ *   q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw: as csa_sparse_attn (shared)
+ * layers * B * Tq <= 65535 (CSA_ERR_UNSUPPORTED_SHAPE otherwise).
+ * ws: csa_workspace_size(CSA_OP_SPARSE_ATTN, layers * B, Tq, n_max). */
+csa_status_t csa_reuse_attn(const csa_params_t* p, csa_dtype_t dtype, int32_t layers,
+                            const void* q, const int32_t* q_pos, const void* kv_cmp,
+                            const int32_t* idx, int32_t n_max, const void* kv_raw,
+                            const int32_t* raw_pos0, const int32_t* n_raw, int32_t raw_max,
+                            const float* sink, int32_t B, int32_t Tq, void* out, void* ws,
+                            size_t ws_bytes, void* stream);
+
 /* Step 4 - HCA dense shared-KV attention ("dense shared-KV attention over all
  * of them plus a 128-token window"): as csa_sparse_attn with the selected
  * set replaced by every visible entry j < n_cmp[b] (p->width, p->stride give

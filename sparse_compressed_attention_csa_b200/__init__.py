@@ -12,12 +12,12 @@ from ._lib import (  # noqa: F401
     CSA_OP_TOPK_SELECT, CsaError, Params, csa_compress, csa_compress_append, csa_index_scores,
     csa_index_topk,
     csa_index_topk_noalloc, csa_last_device_error_site, csa_launch_count, csa_poll_device_error,
-    csa_quantize_fp8, csa_set_wait_limit_ns, csa_sparse_attn, csa_sparse_attn_fp8, csa_topk_select,
+    csa_quantize_fp8, csa_reuse_attn, csa_set_wait_limit_ns, csa_sparse_attn, csa_sparse_attn_fp8, csa_topk_select,
     csa_workspace_size, hca_attn, hca_attn_fp8, lib)
 
 __all__ = [
     "Params", "CsaError", "csa_compress", "csa_compress_append", "csa_index_scores", "csa_topk_select",
     "csa_index_topk", "csa_index_topk_noalloc", "csa_sparse_attn", "hca_attn", "csa_workspace_size",
     "csa_poll_device_error", "csa_last_device_error_site", "csa_set_wait_limit_ns",
-    "csa_launch_count", "csa_quantize_fp8", "csa_sparse_attn_fp8", "hca_attn_fp8", "lib",
+    "csa_launch_count", "csa_quantize_fp8", "csa_reuse_attn", "csa_sparse_attn_fp8", "hca_attn_fp8", "lib",
 ]

@@ -102,6 +102,7 @@ def _load():
     lib.csa_sparse_attn.argtypes = [_PP, ctypes.c_int, _P, _P, _P, _P, _I, _P, _P, _P, _I, _P,
                                     _I, _I, _P, _P, ctypes.c_size_t, _P]
     lib.hca_attn.argtypes = list(lib.csa_sparse_attn.argtypes)
+    lib.csa_reuse_attn.argtypes = [_PP, ctypes.c_int, _I] + list(lib.csa_sparse_attn.argtypes[2:])
     lib.csa_quantize_fp8.argtypes = [ctypes.c_int, _P, ctypes.c_int64, _I, _P, _P, _P]
     lib.csa_sparse_attn_fp8.argtypes = [_PP, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _P, _I,
                                         _I, _P, _P, ctypes.c_size_t, _P]
@@ -118,6 +119,7 @@ def _load():
     for f in ("csa_workspace_size", "csa_compress", "csa_index_scores", "csa_topk_select",
               "csa_index_topk", "csa_sparse_attn", "hca_attn", "csa_poll_device_error",
               "csa_compress_append", "csa_quantize_fp8", "csa_sparse_attn_fp8", "hca_attn_fp8",
+              "csa_reuse_attn",
               "csa_index_topk_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -296,6 +298,29 @@ def csa_sparse_attn(p: Params, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, s
     _req(idx, "idx", torch.int32, 3)
     _attn(_load().csa_sparse_attn, p, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out,
           ws, stream)
+
+
+def csa_reuse_attn(p: Params, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out, ws=None,
+                   stream=None):
+    """CSA2 Reuse layers: q [R][B][Tq][H][d], sink [R][H] -> out [R][B][Tq][H][d],
+    every layer over the same entries, selection (idx [B][Tq][topk]) and window."""
+    import torch
+    _req(q, "q", ndim=5)
+    _req(q_pos, "q_pos", torch.int32, 2)
+    _req(kv_cmp, "kv_cmp", q.dtype, 3)
+    _req(idx, "idx", torch.int32, 3)
+    _req(kv_raw, "kv_raw", q.dtype, 3)
+    _req(raw_pos0, "raw_pos0", torch.int32, 1)
+    _req(n_raw, "n_raw", torch.int32, 1)
+    _req(sink, "sink", torch.float32, 2)
+    _req(out, "out", q.dtype, 5)
+    R = q.shape[0]
+    B, Tq = q_pos.shape
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().csa_reuse_attn(ctypes.byref(p.c()), _dtype_code(q), R, _ptr(q), _ptr(q_pos),
+                                  _ptr(kv_cmp), _ptr(idx), kv_cmp.shape[1], _ptr(kv_raw),
+                                  _ptr(raw_pos0), _ptr(n_raw), kv_raw.shape[1], _ptr(sink), B, Tq,
+                                  _ptr(out), _ptr(ws), nb, _stream(stream)))
 
 
 def hca_attn(p: Params, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, sink, out, ws=None,

@@ -106,6 +106,8 @@ struct AttnPairArgs {
   int raw_max;
   const float* sink;
   int Tq, topk, window, width, stride, rope_dim;
+  int rows_per_layer;  // B * Tq: grid row y is layer y / rows_per_layer (own q, sink, out)
+                       // of token y % rows_per_layer (shared entries, selection, window)
   float scale_log2;
   int splits;
   unsigned long long wait_ns;  // limit of every bounded wait
@@ -248,7 +250,9 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
   const uint32_t peer = rank ^ 1u;
   const int part = (int)rank;
   const int split = (int)(blockIdx.x >> 1);
-  const int row_q = blockIdx.y;  // b * Tq + tq
+  const int row_all = blockIdx.y;               // layer * B * Tq + b * Tq + tq
+  const int row_q = row_all % a.rows_per_layer;  // b * Tq + tq: entries, selection, window
+  const int layer = row_all / a.rows_per_layer;  // q, sink and out of this layer
   const int b = row_q / a.Tq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rope0 = kApDim - a.rope_dim;
@@ -301,7 +305,8 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
     tma_prefetch_desc(&tm_raw);
     mbar_arrive_expect_tx(&sm.q_tma, kApHeads * kApHalf * 2);
     for (int sb = 0; sb < 4; ++sb)
-      tma_load_2d(q_stage + sb * kApSubBytes, &tm_q, &sm.q_tma, dim0 + sb * 64, row_q * kApHeads);
+      tma_load_2d(q_stage + sb * kApSubBytes, &tm_q, &sm.q_tma, dim0 + sb * 64,
+                  row_all * kApHeads);
   }
   if (warp == 8) {
     // RoPE table at the query position
@@ -624,7 +629,7 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
       if (S == 1) {
         // normalise with the sink, rotate the output's RoPE dims back by -t,
         // bf16, TMA store of 32-dim boxes ([128 heads][64 B], 64B swizzle)
-        const float sink_l2 = a.sink[head] * 1.4426950408889634f;
+        const float sink_l2 = a.sink[layer * kApHeads + head] * 1.4426950408889634f;
         const float mm = fmaxf(m_run, sink_l2);
         const float den = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - mm)) +
                           exp2f(sink_l2 - mm);
@@ -667,7 +672,7 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (threadIdx.x == 0) {
           for (int sl = 0; sl < kApSlabs; ++sl)
-            tma_store_2d(&tm_out, ring + sl * kApOutBoxBytes, dim0 + sl * 32, row_q * kApHeads);
+            tma_store_2d(&tm_out, ring + sl * kApOutBoxBytes, dim0 + sl * 32, row_all * kApHeads);
           bulk_commit();
           bulk_wait_read_all();
         }
@@ -676,7 +681,7 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
         // k_attn_merge (values of order one: fp16 keeps 11 bits).  O leaves
         // through the ring as 8 contiguous 8 KB slabs ([16-byte unit u][head]
         // [8 halves] per 32 dims) and one bulk copy.
-        const size_t unit = ((size_t)row_q * S + split) * 2 + part;
+        const size_t unit = ((size_t)row_all * S + split) * 2 + part;
         float* pml = a.part_ml + unit * 2 * kApHeads;
         pml[head] = m_run;
         pml[kApHeads + head] = l_run;
@@ -956,6 +961,7 @@ struct AttnMergeArgs {
   const int* q_pos;
   int splits;
   int rope_dim;
+  int rows_per_layer;  // as in AttnPairArgs
   __nv_bfloat16* out;
   double freq[kApMaxRope / 2];
 };
@@ -965,7 +971,8 @@ __global__ void __launch_bounds__(kApHeads) k_attn_merge(AttnMergeArgs a) {
   sm100::griddep_wait();  // the partials of the attention kernel are visible
   sm100::griddep_launch_dependents();
   const int part = blockIdx.x >> 3, sl = blockIdx.x & 7;
-  const int row_q = blockIdx.y;
+  const int row_all = blockIdx.y;  // layer * rows_per_layer + token
+  const int row_q = row_all % a.rows_per_layer, layer = row_all / a.rows_per_layer;
   const int head = threadIdx.x;
   const int S = a.splits;
   const int rope0 = kApDim - a.rope_dim;
@@ -980,7 +987,7 @@ __global__ void __launch_bounds__(kApHeads) k_attn_merge(AttnMergeArgs a) {
       sn[head] = s;
     }
   }
-  const size_t unit0 = (size_t)row_q * S * 2 + part;  // unit of split s: unit0 + 2 s
+  const size_t unit0 = (size_t)row_all * S * 2 + part;  // unit of split s: unit0 + 2 s
   auto slab_of = [&](int s) {
     return reinterpret_cast<const uint4*>(a.part_o + (unit0 + 2 * (size_t)s) * kApHeads * kApHalf) +
            (size_t)sl * (kApSlabBytes / 16);
@@ -1003,7 +1010,7 @@ __global__ void __launch_bounds__(kApHeads) k_attn_merge(AttnMergeArgs a) {
 #pragma unroll
     for (int u = 0; u < 4; ++u)
       x[j][u] = j < S ? __ldcg(slab_of(j) + u * kApHeads + head) : make_uint4(0u, 0u, 0u, 0u);
-  const float sink_l2 = a.sink[head] * 1.4426950408889634f;
+  const float sink_l2 = a.sink[layer * kApHeads + head] * 1.4426950408889634f;
   float M = sink_l2;
 #pragma unroll
   for (int s = 0; s < kApMaxSplits; ++s) M = fmaxf(M, mv[s]);
@@ -1057,7 +1064,7 @@ __global__ void __launch_bounds__(kApHeads) k_attn_merge(AttnMergeArgs a) {
       }
     }
   }
-  uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)row_q * kApHeads + head) * kApDim + d0);
+  uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)row_all * kApHeads + head) * kApDim + d0);
 #pragma unroll
   for (int u = 0; u < 4; ++u)
     dst[u] = make_uint4(ap_bf16x2(o[8 * u], o[8 * u + 1]), ap_bf16x2(o[8 * u + 2], o[8 * u + 3]),

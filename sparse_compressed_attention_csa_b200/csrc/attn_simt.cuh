@@ -30,6 +30,7 @@ struct AttnArgs {
   const float* sink;
   const float* cmp_scale;  // FP8 caches (tensor-core path only): row scales
   const float* raw_scale;
+  int layers;  // tensor-core path: layers sharing entries and selection (q, sink, out per layer)
   int B, Tq, H, d, rope_dim, topk, window, width, stride;
   float scale;  // with the extended RoPE's temperature
   RopeSpec rope;

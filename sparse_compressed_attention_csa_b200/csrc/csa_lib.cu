@@ -788,8 +788,9 @@ static csa_status_t launch_attn_simt(const AttnArgs& a, csa_dtype_t dtype, cudaS
 template <bool kHca, bool kFp8 = false>
 static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, void* ws,
                                    size_t ws_bytes, cudaStream_t s) {
-  const int sp = attn_splits(p, kHca, g.B, g.Tq, g.n_max);
-  const size_t need = attn_ws_bytes(p, CSA_BF16, kHca, g.B, g.Tq, g.n_max);
+  const int LB = g.layers * g.B;  // (layer, sequence) rows of the grid
+  const int sp = attn_splits(p, kHca, LB, g.Tq, g.n_max);
+  const size_t need = attn_ws_bytes(p, CSA_BF16, kHca, LB, g.Tq, g.n_max);
   if (ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes, need %zu", ws_bytes, need);
   if (need > 0) CSA_CHECK(check_ptr(ws, "ws"));
@@ -808,6 +809,7 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   a.raw_max = g.raw_max;
   a.sink = g.sink;
   a.Tq = g.Tq;
+  a.rows_per_layer = g.B * g.Tq;
   a.topk = g.topk;
   a.window = g.window;
   a.width = g.width;
@@ -821,15 +823,15 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   a.part_ml = nullptr;
   if (sp > 1) {
     // workspace: partial O | partial (m, l)
-    const size_t units = (size_t)g.B * g.Tq * sp * 2;
+    const size_t units = (size_t)LB * g.Tq * sp * 2;
     const size_t o_bytes = round_up(units * kApHeads * kApHalf * sizeof(__half), 256);
     a.part_o = (__half*)ws;
     a.part_ml = (float*)((char*)ws + o_bytes);
   }
   for (int i = 0; i < kApMaxRope / 2; ++i) a.freq[i] = i < g.rope_dim / 2 ? rope_freq(g.rope, i) : 0.0;
   CUtensorMap tq, to, tc, tr;
-  CSA_CHECK(make_tmap_bf16(&tq, g.q, kApDim, (uint64_t)g.B * g.Tq * kApHeads, 64, kApHeads));
-  CSA_CHECK(make_tmap_bf16(&to, g.out, kApDim, (uint64_t)g.B * g.Tq * kApHeads, 32, kApHeads,
+  CSA_CHECK(make_tmap_bf16(&tq, g.q, kApDim, (uint64_t)LB * g.Tq * kApHeads, 64, kApHeads));
+  CSA_CHECK(make_tmap_bf16(&to, g.out, kApDim, (uint64_t)LB * g.Tq * kApHeads, 32, kApHeads,
                            CU_TENSOR_MAP_SWIZZLE_64B));
   // row gathers (one-row boxes of 64 dims); a cache with no rows is never
   // read, and its map is made over q instead
@@ -847,7 +849,7 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
                              n_raw_rows ? n_raw_rows : n_q_rows, 64, 1));
   }
   CSA_CHECK(set_smem_attr(k_attn_pair<kHca, kFp8>, kApSmemBytes, "k_attn_pair"));
-  dim3 grid((unsigned)(2 * sp), (unsigned)(g.B * g.Tq));
+  dim3 grid((unsigned)(2 * sp), (unsigned)(LB * g.Tq));
   cudaError_t e = launch_ex(k_attn_pair<kHca, kFp8>, grid,
                             dim3(kFp8 ? kApThreadsFp8 : kApThreads), kApSmemBytes, s, 2, a, tq, to,
                             tc, tr);
@@ -861,9 +863,10 @@ static csa_status_t launch_attn_tc(const csa_params_t* p, const AttnArgs& g, voi
   m.q_pos = g.q_pos;
   m.splits = sp;
   m.rope_dim = g.rope_dim;
+  m.rows_per_layer = g.B * g.Tq;
   m.out = a.out;
   for (int i = 0; i < kApMaxRope / 2; ++i) m.freq[i] = a.freq[i];
-  e = launch_ex(k_attn_merge, dim3(2 * kApSlabs, (unsigned)(g.B * g.Tq)), dim3(kApHeads), 0, s, 1,
+  e = launch_ex(k_attn_merge, dim3(2 * kApSlabs, (unsigned)(LB * g.Tq)), dim3(kApHeads), 0, s, 1,
                 m);
   if (e != cudaSuccess) return cuda_fail(e, "k_attn_merge");
   return launched("k_attn_merge");
@@ -877,7 +880,7 @@ static AttnArgs make_attn_args(const csa_params_t* p, const void* q, const int32
   AttnArgs a;
   a.q = q; a.q_pos = q_pos; a.kv_cmp = kv_cmp; a.idx = idx; a.n_cmp = n_cmp; a.n_max = n_max;
   a.kv_raw = kv_raw; a.raw_pos0 = raw_pos0; a.n_raw = n_raw; a.raw_max = raw_max; a.sink = sink;
-  a.cmp_scale = nullptr; a.raw_scale = nullptr;
+  a.cmp_scale = nullptr; a.raw_scale = nullptr; a.layers = 1;
   a.B = B; a.Tq = Tq; a.H = p->n_heads; a.d = p->d; a.rope_dim = p->rope_dim; a.topk = p->topk;
   a.window = p->window; a.width = p->width; a.stride = p->stride; a.scale = attn_scale(p);
   a.rope = rope_spec(p); a.out = out;
@@ -900,6 +903,40 @@ CSA_API csa_status_t csa_sparse_attn(const csa_params_t* p, csa_dtype_t dtype, c
   if (attn_tc_ok(p, dtype, false, n_max))
     return launch_attn_tc<false>(p, a, ws, ws_bytes, (cudaStream_t)stream);
   return launch_attn_simt<false>(a, dtype, (cudaStream_t)stream);
+}
+
+CSA_API csa_status_t csa_reuse_attn(const csa_params_t* p, csa_dtype_t dtype, int32_t layers,
+                                    const void* q, const int32_t* q_pos, const void* kv_cmp,
+                                    const int32_t* idx, int32_t n_max, const void* kv_raw,
+                                    const int32_t* raw_pos0, const int32_t* n_raw,
+                                    int32_t raw_max, const float* sink, int32_t B, int32_t Tq,
+                                    void* out, void* ws, size_t ws_bytes, void* stream) {
+  CSA_CHECK(attn_common_checks(p, dtype, q, q_pos, kv_cmp, n_max, kv_raw, raw_pos0, n_raw,
+                               raw_max, sink, B, Tq, out));
+  CSA_CHECK(check_topk(p));
+  CSA_CHECK(check_ptr(idx, "idx"));
+  if (layers < 1 || (long long)layers * B * Tq > 65535)
+    return fail(CSA_ERR_UNSUPPORTED_SHAPE, "layers=%d x B*Tq=%d beyond 65535 query rows", layers,
+                B * Tq);
+  CSA_CHECK(check_device());
+  AttnArgs a = make_attn_args(p, q, q_pos, kv_cmp, idx, nullptr, n_max, kv_raw, raw_pos0, n_raw,
+                              raw_max, sink, B, Tq, out);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (attn_tc_ok(p, dtype, false, n_max)) {
+    a.layers = layers;
+    return launch_attn_tc<false>(p, a, ws, ws_bytes, s);
+  }
+  // generic path: one launch per layer
+  const size_t esz = dtype == CSA_BF16 ? 2 : 4;
+  const size_t per = (size_t)B * Tq * p->n_heads * p->d * esz;
+  for (int r = 0; r < layers; ++r) {
+    AttnArgs ar = a;
+    ar.q = (const char*)q + r * per;
+    ar.out = (char*)out + r * per;
+    ar.sink = sink + (size_t)r * p->n_heads;
+    CSA_CHECK(launch_attn_simt<false>(ar, dtype, s));
+  }
+  return CSA_OK;
 }
 
 CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const void* q,

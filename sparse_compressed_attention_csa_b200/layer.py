@@ -81,17 +81,25 @@ def hca_decode(p: L.Params, q, q_pos, kv_cmp, n_cmp, kv_raw, raw_pos0, n_raw, si
 
 def reuse_attn(p: L.Params, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink,
                ws: Workspace | None = None, out=None, stream=None):
-    """A Reuse layer of CSA2 ("CSA2 encoder layers (2x compression, Full +
-    Reuse)": the rest reuse that KV and its top-512 selection): this layer's
-    queries and sink over the entries and indices a Full layer produced."""
+    """Reuse layers of CSA2 ("CSA2 encoder layers (2x compression, Full +
+    Reuse)": the rest reuse that KV and its top-512 selection): each layer's
+    queries q [R][B][Tq][H][d] and sink [R][H] over the entries and indices a
+    Full layer produced, all R layers in one call (a single layer:
+    q [B][Tq][H][d], sink [H])."""
     ws = ws or Workspace(q.device)
-    B, Tq = q_pos.shape
+    single = q.dim() == 4
+    if single:
+        q, sink = q.unsqueeze(0), sink.unsqueeze(0)
     if out is None:
         out = torch.empty_like(q)
-    nb = L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, B, Tq, kv_cmp.shape[1])
-    L.csa_sparse_attn(p, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out, ws.get(nb),
-                      stream)
-    return out
+    elif single:
+        out = out.unsqueeze(0)
+    R = q.shape[0]
+    B, Tq = q_pos.shape
+    nb = L.csa_workspace_size(p, L.CSA_OP_SPARSE_ATTN, R * B, Tq, kv_cmp.shape[1])
+    L.csa_reuse_attn(p, q, q_pos, kv_cmp, idx, kv_raw, raw_pos0, n_raw, sink, out, ws.get(nb),
+                     stream)
+    return out[0] if single else out
 
 
 def hca_prefill(p: L.Params, x, gate, q, sink, ws: Workspace | None = None, out=None,

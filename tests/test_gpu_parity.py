@@ -205,7 +205,7 @@ def test_prefill_extended_rope_small_original_context():
 def test_csa2_full_and_reuse_layers():
     # 2 -> 1 pooling, top-512, YaRN; the Reuse layers attend with their own
     # queries and sinks over the Full layer's entries and selection
-    wl = W.CSA2_DECODE.replace(B=3, T=20001, reuse_layers=2, seed=46)
+    wl = W.CSA2_DECODE.replace(B=3, T=20001, reuse_layers=3, seed=46)
     data = W.generate(wl)
     idx, out = run_decode(wl, data)
     seqs = list(range(wl.B))
@@ -214,16 +214,21 @@ def test_csa2_full_and_reuse_layers():
     assert_close(host64(out), out_o, wl.dtype, wl.name)
     p = params_of(wl)
     t = {k: dev(data[k]) for k in ("q_pos", "kv_cmp", "kv_raw", "raw_pos0", "n_raw")}
+    # every Reuse layer in one call, and layer 1 alone
+    o_all = layer.reuse_attn(p, dev(data["q_reuse"]), t["q_pos"], t["kv_cmp"], idx, t["kv_raw"],
+                             t["raw_pos0"], t["n_raw"], dev(data["sink_reuse"]))
+    o_one = layer.reuse_attn(p, dev(data["q_reuse"][1]), t["q_pos"], t["kv_cmp"], idx,
+                             t["kv_raw"], t["raw_pos0"], t["n_raw"], dev(data["sink_reuse"][1]))
+    torch.cuda.synchronize()
     for r in range(wl.reuse_layers):
-        o = layer.reuse_attn(p, dev(data["q_reuse"][r]), t["q_pos"], t["kv_cmp"], idx,
-                             t["kv_raw"], t["raw_pos0"], t["n_raw"], dev(data["sink_reuse"][r]))
-        torch.cuda.synchronize()
         want = np.stack([oracle.sparse_attn(
             f64(data, "q_reuse", r, b),
             data["q_pos"][b], _vals(data["kv_cmp"][b]), idx_o[b], _vals(data["kv_raw"][b]),
             int(data["raw_pos0"][b]), int(data["n_raw"][b]), data["sink_reuse"][r], wl.scale,
             wl.window, wl.rope_dim, theta_of(wl)) for b in seqs])
-        assert_close(host64(o), want, wl.dtype, f"{wl.name} reuse layer {r}")
+        assert_close(host64(o_all[r]), want, wl.dtype, f"{wl.name} reuse layer {r}")
+        if r == 1:
+            assert_close(host64(o_one), want, wl.dtype, f"{wl.name} reuse layer 1 alone")
 
 
 def test_decode_context_too_short_for_any_entry():
