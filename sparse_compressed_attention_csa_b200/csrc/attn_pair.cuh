@@ -25,9 +25,11 @@
 //
 //   warp 8 (one thread): MMAs   S(i) = Q K_i^T (N = 64, K = 256, A from TMEM)
 //                               O   += P(j) V(j) (N = 256, A = P from TMEM)
-//   warps 4-7: q by TMA, the row list, then the gather: TMA tile::gather4
-//              (four rows x 64 dims per instruction) of the CTA's half of
-//              each row into 128B-swizzled chunks.  A gather4 holds its
+//   warps 4-7: q by TMA, the row list (the window's rows first: their
+//              leading tiles are gathered while the selection's indices
+//              load), then the gather: TMA tile::gather4 (four rows x 64
+//              dims per instruction) of the CTA's half of each row into
+//              128B-swizzled chunks.  A gather4 holds its
 //              warp for ~60 ns (one warp moves ~16 GB/s), so four warps
 //              issue: warp 4 + (2 (i % 2) + c) fetches chunk c of tile i.
 //   warps 0-3: one head per thread (= TMEM lane): this CTA's partial logits
@@ -127,8 +129,8 @@ struct ApMisc {
   uint64_t q_tma, q_ready, rows_ready, rope_ready, mma_drain;
   uint32_t tmem_base;
   int n_rows;  // padded rows (multiple of 4)
-  int n_sel;   // selected rows (valid rows [0, n_sel))
-  int n_win;   // window rows (valid rows [pad4(n_sel), pad4(n_sel) + n_win))
+  int n_win;   // window rows (valid rows [0, n_win))
+  int n_sel;   // selected / visible entries (valid rows [pad4(n_win), pad4(n_win) + n_sel))
   int abort_flag;
   int scan_tmp[4];
   int last_n[kApSlots];  // last chunk requested into each ring slot (-1: none)
@@ -319,39 +321,119 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
     mbar_arrive(&sm.rope_ready);
   }
 
+  // The row list: the window's raw rows (padded to a multiple of 4), then
+  // the selected (or, for HCA, every visible) entries in their order (padded
+  // likewise).  Global tile t (64 rows of the list) belongs to split t % S:
+  // this CTA's tile i is global tile split + i * S, so the window's tiles,
+  // known without the selection, lead the first splits.
+  auto tile_row0 = [&](int i) { return (split + i * S) * kApTile; };
+
+  // One chunk's gathers (the slot is free): bf16 rows, lane l fetches rows
+  // 4 (l & 15) .. + 3 of the tile, 64-dim half l >> 4; groups at or past
+  // n_rows are zero-filled, so that masked rows hold finite values.
+  auto gather_chunk_bf16 = [&](int i, int ck, int n_rows, int pw) {
+    const int n = 2 * i + ck;
+    const int slot = n % kApSlots;
+    const int h = lane >> 4, rg = lane & 15;
+    const int g = tile_row0(i) + 4 * rg;  // list index of the group's first row
+    const bool valid = g < n_rows;
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    uint8_t* dst = ring + slot * kApChunkBytes + h * (kApChunkBytes / 2) + rg * 512;
+    if (!valid) {
+#pragma unroll
+      for (int u = 0; u < 32; ++u) reinterpret_cast<uint4*>(dst)[u] = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_shared();  // read by the MMA (async proxy)
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)__popc(vmask) * 512u);
+      sm.last_n[slot] = n;
+    }
+    if (valid)
+      tma_gather4(dst, g < pw ? &tm_raw : &tm_cmp, &sm.full[slot], dim0 + ck * 128 + h * 64,
+                  sm.rows[g], sm.rows[g + 1], sm.rows[g + 2], sm.rows[g + 3]);
+  };
+  // FP8: lanes 0-15 each gather the codes of rows 4l .. 4l + 3 (128 B a row)
+  // into the upper half of the slot; the rows' scales go to sm.scl.
+  auto gather_chunk_fp8 = [&](int i, int ck, int n_rows, int pw) {
+    const int n = 2 * i + ck;
+    const int slot = n % kApSlots;
+    const int g0 = tile_row0(i);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int gi = g0 + lane + 32 * q;
+      sm.scl[slot][lane + 32 * q] =
+          gi < n_rows ? (gi < pw ? a.raw_scale : a.cmp_scale)[sm.rows[gi]] : 0.f;
+    }
+    const int g = g0 + 4 * lane;
+    const bool gv = lane < 16 && g < n_rows;
+    const unsigned vmask = __ballot_sync(0xffffffffu, gv);  // also orders the scales
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.stage[slot], (uint32_t)__popc(vmask) * 512u);
+      sm.last_n[slot] = n;
+    }
+    __syncwarp();
+    if (gv)
+      tma_gather4(ring + slot * kApChunkBytes + kApChunkBytes / 2 + lane * 512,
+                  g < pw ? &tm_raw : &tm_cmp, &sm.stage[slot], dim0 + ck * 128, sm.rows[g],
+                  sm.rows[g + 1], sm.rows[g + 2], sm.rows[g + 3]);
+  };
+
+  int early = 0;  // warps 4-7: this CTA's leading tiles already gathered from the window
   if (warp >= 4 && warp < 8) {
-    // ======================= row list (warps 4-7): gather coordinates of the
-    // selected (or visible) entries in their order, then the window's raw
-    // rows, each part padded to a multiple of 4 rows.  Both CTAs of a pair
-    // build the same list.
+    // ======================= row list (warps 4-7); both CTAs of a pair
+    // build the same list.  CSA: the selection's entries are loaded first;
+    // the window part is written and its leading tiles gathered while the
+    // loads are in flight, then the selection is placed after it.
     const int tid = threadIdx.x - 128;
     const int cmp_y0 = b * a.n_max;
     const int raw_y0 = b * a.raw_max;
-    const int rp0 = a.raw_pos0[b];
-    const int nraw = a.n_raw[b];
-    int n_sel;
-    if (kHca) {
-      const int nv = min(min(n_visible(t, a.n_cmp[b], a.width, a.stride), a.n_max), kApRowCap);
-      for (int j = tid; j < nv; j += 128) sm.rows[j] = cmp_y0 + j;
-      n_sel = nv;
-    } else {
-      // thread tid compacts entries [tid * E, tid * E + E) of the selection;
-      // one block scan of the valid counts places them
+    constexpr int kMaxE = kApRowCap / 128;
+    int jv[kMaxE];
+    const int E = kHca ? 0 : (a.topk + 127) / 128;
+    if (!kHca) {
+      // thread tid compacts entries [tid * E, tid * E + E) of the selection
       const int* sel = a.idx + (size_t)row_q * a.topk;
-      constexpr int kMaxE = kApRowCap / 128;
-      const int E = (a.topk + 127) / 128;
-      int jv[kMaxE];
-      int cnt = 0;
 #pragma unroll
       for (int e = 0; e < kMaxE; ++e) {
         const int i = tid * E + e;
-        int j = (e < E && i < a.topk) ? sel[i] : -1;
-        if (j >= a.n_max) {
+        jv[e] = (e < E && i < a.topk) ? sel[i] : -1;
+      }
+    }
+    const int rp0 = a.raw_pos0[b];
+    const int nraw = a.n_raw[b];
+    const int w_lo = max(max(0, t - a.window + 1), rp0);
+    const int w_hi = min(t, rp0 + min(nraw, a.raw_max) - 1);
+    int n_win = (a.window > 0 && w_hi >= w_lo) ? w_hi - w_lo + 1 : 0;
+    n_win = max(0, min(n_win, kApRowCap));
+    const int pw = (n_win + 3) & ~3;
+    for (int u = tid; u < pw; u += 128)
+      sm.rows[u] = raw_y0 + (w_lo - rp0) + (u < n_win ? u : 0);
+    int n_sel = 0;
+    if (kHca) {
+      n_sel = min(min(n_visible(t, a.n_cmp[b], a.width, a.stride), a.n_max), kApRowCap - pw);
+      for (int j = tid; j < n_sel; j += 128) sm.rows[pw + j] = cmp_y0 + j;
+    } else {
+      asm volatile("bar.sync 2, 128;" ::: "memory");  // window rows written
+      // leading tiles of window rows only, gathered before the selection is
+      // placed: at most 3, whose chunks take ring slots 0-5 for the first
+      // time (no wait on a slot or on the q staging)
+      while (early < 3 && tile_row0(early) + kApTile <= pw) ++early;
+      if (kFp8) {
+        if (warp < 6)
+          for (int i = 0; i < early; ++i) gather_chunk_fp8(i, warp - 4, pw, pw);
+      } else {
+        for (int i = (warp - 4) >> 1; i < early; i += 2) gather_chunk_bf16(i, (warp - 4) & 1, pw, pw);
+      }
+      // the selection: one block scan of the valid counts places it
+      int cnt = 0;
+#pragma unroll
+      for (int e = 0; e < kMaxE; ++e) {
+        if (jv[e] >= a.n_max) {
           report_error(CSA_ERR_DEVICE_BOUNDS);
-          j = -1;
+          jv[e] = -1;
         }
-        jv[e] = j;
-        cnt += j >= 0 ? 1 : 0;
+        cnt += jv[e] >= 0 ? 1 : 0;
       }
       int x = cnt;
 #pragma unroll
@@ -368,45 +450,36 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
         off += w < warp - 4 ? c : 0;
         tot += c;
       }
+      const int cap = kApRowCap - pw;
 #pragma unroll
       for (int e = 0; e < kMaxE; ++e) {
         if (jv[e] >= 0) {
-          if (off < kApRowCap) sm.rows[off] = cmp_y0 + jv[e];
+          if (off < cap) sm.rows[pw + off] = cmp_y0 + jv[e];
           ++off;
         }
       }
-      n_sel = min(tot, kApRowCap);
+      n_sel = min(tot, cap);
     }
     const int ps = (n_sel + 3) & ~3;
-    for (int k = n_sel + tid; k < ps; k += 128) sm.rows[k] = cmp_y0;  // masked padding
-    {
-      const int w_lo = max(max(0, t - a.window + 1), rp0);
-      const int w_hi = min(t, rp0 + min(nraw, a.raw_max) - 1);
-      int n_win = (a.window > 0 && w_hi >= w_lo) ? w_hi - w_lo + 1 : 0;
-      n_win = max(0, min(n_win, kApRowCap - ps));
-      const int pw = (n_win + 3) & ~3;
-      for (int u = tid; u < pw; u += 128)
-        sm.rows[ps + u] = raw_y0 + (w_lo - rp0) + (u < n_win ? u : 0);
-      if (tid == 0) {
-        sm.n_sel = n_sel;
-        sm.n_win = n_win;
-        sm.n_rows = ps + pw;
-      }
+    for (int k = n_sel + tid; k < ps; k += 128) sm.rows[pw + k] = cmp_y0;  // masked padding
+    if (tid == 0) {
+      sm.n_sel = n_sel;
+      sm.n_win = n_win;
+      sm.n_rows = pw + ps;
     }
     asm volatile("bar.sync 2, 128;" ::: "memory");  // rows written
     mbar_arrive(&sm.rows_ready);
   }
 
-  // this split's rows, in groups of 4 (each role waits for rows_ready
-  // before reading the list); the two CTAs of a pair take the same rows
+  // this split's tiles (each role waits for rows_ready before reading the
+  // list); the two CTAs of a pair take the same rows
   bool rows_ok = false;
-  int r_lo = 0, r_hi = 0, ntile = 0;
+  int n_rows = 0, ntile = 0;
   auto load_split = [&]() {
     rows_ok = mbar_wait(&sm.rows_ready, 0, abortp, wait_ns);
-    const int G = rows_ok ? sm.n_rows / 4 : 0;
-    r_lo = 4 * (int)((long long)G * split / S);
-    r_hi = 4 * (int)((long long)G * (split + 1) / S);
-    ntile = (r_hi - r_lo + kApTile - 1) / kApTile;
+    n_rows = rows_ok ? sm.n_rows : 0;
+    const int tiles = (n_rows + kApTile - 1) / kApTile;
+    ntile = tiles > split ? (tiles - split + S - 1) / S : 0;
   };
 
   // exchange bookkeeping of thread 0: partner tiles whose 16 KB this CTA
@@ -478,7 +551,8 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
     // read tile i from that buffer (each thread reads tile i before it sends
     // tile i + 1).  (Sending one tile ahead of the softmax instead measured
     // slower: with two S buffers the next QK is not ready in time.)
-    const int n_sel = sm.n_sel, ps = (n_sel + 3) & ~3, pe = ps + sm.n_win;
+    // valid rows: the window's [0, n_win) and the entries' [pw, pe)
+    const int nw = sm.n_win, pw = (nw + 3) & ~3, pe = pw + sm.n_sel;
     for (int i = 0; i < ntile && ok; ++i) {
       const int sb = i & 1;
       const int xb = i % kApXBufs;
@@ -543,13 +617,13 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
       // rows of the tile outside the split, padding between the selected and
       // the window rows, and padding at the end are masked; most tiles have
       // none
-      const int g0 = r_lo + i * kApTile;  // list index of row 0 of the tile
+      const int g0 = tile_row0(i);  // list index of row 0 of the tile
       const int g1 = g0 + kApTile - 1;
-      if (!(g1 < r_hi && (g1 < n_sel || (g0 >= ps && g1 < pe)))) {
+      if (!(g1 < n_rows && (g1 < nw || (g0 >= pw && g1 < pe)))) {
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const int g = g0 + e;
-          const bool valid = g < r_hi && (g < n_sel || (g >= ps && g < pe));
+          const bool valid = g < n_rows && (g < nw || (g >= pw && g < pe));
           if (!valid) z[e] = -INFINITY;
         }
       }
@@ -730,11 +804,11 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
     load_split();
     const int ex = warp < 8 ? warp - 6 : warp - 7;  // expander index (warps 6, 7, 9, 10)
     const int ck = warp < 6 ? warp - 4 : ex & 1;
-    const int ps = (sm.n_sel + 3) & ~3;
+    const int pw = (sm.n_win + 3) & ~3;
     bool okp = __all_sync(0xffffffffu, rows_ok);
     if (warp < 6) {
       bool staged = false;  // q staging slots handed back
-      for (int i = 0; i < ntile && okp; ++i) {
+      for (int i = early; i < ntile && okp; ++i) {  // the first `early` went out with the list
         const int n = 2 * i + ck;
         const int slot = n % kApSlots;
         if (lane == 0) {
@@ -746,25 +820,7 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
         }
         okp = __shfl_sync(0xffffffffu, okp ? 1 : 0, 0) != 0;
         if (!okp) break;
-        const int g0 = r_lo + i * kApTile;  // list index of the chunk's row 0
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int gi = g0 + lane + 32 * q;
-          sm.scl[slot][lane + 32 * q] =
-              gi < r_hi ? (gi < ps ? a.cmp_scale : a.raw_scale)[sm.rows[gi]] : 0.f;
-        }
-        const int g = g0 + 4 * lane;
-        const bool gv = lane < 16 && g < r_hi;
-        const unsigned vmask = __ballot_sync(0xffffffffu, gv);  // also orders the scales
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&sm.stage[slot], (uint32_t)__popc(vmask) * 512u);
-          sm.last_n[slot] = n;
-        }
-        __syncwarp();
-        if (gv)
-          tma_gather4(ring + slot * kApChunkBytes + kApChunkBytes / 2 + lane * 512,
-                      g < ps ? &tm_cmp : &tm_raw, &sm.stage[slot], dim0 + ck * 128, sm.rows[g],
-                      sm.rows[g + 1], sm.rows[g + 2], sm.rows[g + 3]);
+        gather_chunk_fp8(i, ck, n_rows, pw);
       }
     } else {
       for (int i = 0; i < ntile && okp; ++i) {
@@ -773,10 +829,10 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
         okp = __all_sync(0xffffffffu, mbar_wait(&sm.stage[slot], (uint32_t)(n / kApSlots) & 1u,
                                                 abortp, wait_ns));
         if (!okp) break;
-        const int g0 = r_lo + i * kApTile;
+        const int g0 = tile_row0(i);
         uint8_t* sl = ring + slot * kApChunkBytes;
         const int r = 32 * (ex >> 1) + lane;
-        if (g0 + r < r_hi)
+        if (g0 + r < n_rows)
           ap_expand_fp8_row(sl, r, sm.scl[slot][r]);
         else
           ap_zero_row(sl, r);
@@ -788,17 +844,16 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
   } else if (warp < 8) {
     // ======================= gather producers (warps 4-7)
     // Chunk n (tile n / 2, dims dim0 + 128 (n % 2)) goes to ring slot
-    // n % kApSlots; warp 4 + (2 (i % 2) + c) fetches chunk c of tile i.
-    // Lane l fetches rows 4 (l & 15) .. + 3 of the tile, 64-dim half l >> 4,
-    // with one gather4.  Groups past the split end (only in its last tile)
-    // are zero-filled, so that masked rows hold finite values.
+    // n % kApSlots; warp 4 + (2 (i % 2) + c) fetches chunk c of tile i with
+    // one gather4 per lane (gather_chunk_bf16).  The first `early` tiles went
+    // out with the row list.
     load_split();
     const int ck = (warp - 4) & 1, tpar = (warp - 4) >> 1;
-    const int h = lane >> 4, rg = lane & 15;
-    const int ps = (sm.n_sel + 3) & ~3;
+    const int pw = (sm.n_win + 3) & ~3;
     bool okp = __all_sync(0xffffffffu, rows_ok);
     bool staged = false;  // q staging slots handed back
     for (int i = tpar; i < ntile && okp; i += 2) {
+      if (i < early) continue;
       const int n = 2 * i + ck;
       const int slot = n % kApSlots;
       if (lane == 0) {
@@ -810,23 +865,7 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
       }
       okp = __shfl_sync(0xffffffffu, okp ? 1 : 0, 0) != 0;
       if (!okp) break;
-      const int g = r_lo + i * kApTile + 4 * rg;  // list index of the group's first row
-      const bool valid = g < r_hi;
-      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-      uint8_t* dst = ring + slot * kApChunkBytes + h * (kApChunkBytes / 2) + rg * 512;
-      if (!valid) {
-#pragma unroll
-        for (int u = 0; u < 32; ++u) reinterpret_cast<uint4*>(dst)[u] = make_uint4(0u, 0u, 0u, 0u);
-        fence_proxy_async_shared();  // read by the MMA (async proxy)
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)__popc(vmask) * 512u);
-        sm.last_n[slot] = n;
-      }
-      if (valid)
-        tma_gather4(dst, g < ps ? &tm_cmp : &tm_raw, &sm.full[slot], dim0 + ck * 128 + h * 64,
-                    sm.rows[g], sm.rows[g + 1], sm.rows[g + 2], sm.rows[g + 3]);
+      gather_chunk_bf16(i, ck, n_rows, pw);
     }
   } else if (warp == 8 && lane == 0) {
     // ======================= MMA issuer

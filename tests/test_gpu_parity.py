@@ -162,15 +162,20 @@ def test_decode_fewer_visible_than_k():
 
 
 def test_decode_running_max_moves_for_some_heads_only():
-    # window row 60 set to 14 x the unit direction of the query of one head
-    # per warp (heads 3, 40, 77, 110; non-rotated dims only): those heads see
-    # a logit of about 13 on it, above their running maximum by more than
-    # the lazy-rescale threshold (2^8), the other heads a small one, so the
-    # lanes of each softmax warp disagree on rescaling O in a late tile.
-    # The row's values stay of order one (the tolerance is absolute).
+    # the last selected entry of each sequence (the list's last tile: window
+    # rows come first, entries after, in index order) set to 14 x the unit
+    # direction of the query of one head per warp (heads 3, 40, 77, 110;
+    # non-rotated dims only): those heads see a logit of about 13 on it,
+    # above their running maximum by more than the lazy-rescale threshold
+    # (2^8), the other heads a small one, so the lanes of each softmax warp
+    # disagree on rescaling O in a late tile.  The row's values stay of order
+    # one (the tolerance is absolute).
     wl = W.CSA_DECODE_64K.replace(B=2, T=5003, seed=47)
     data = W.generate(wl)
-    raw = bits_to_f32(data["kv_raw"]).copy()
+    idx_o = np.stack([oracle.index_topk(f64(data, "q_idx", b), data["w"][b], f64(data, "k_idx", b),
+                                        data["q_pos"][b], int(data["n_cmp"][b]), wl.width,
+                                        wl.stride, wl.topk)[0] for b in range(wl.B)])
+    cmp = bits_to_f32(data["kv_cmp"]).copy()
     q = bits_to_f32(data["q"]).astype(np.float64)  # [B, 1, H, d]
     nr = wl.d - wl.rope_dim
     for b in range(wl.B):
@@ -178,12 +183,12 @@ def test_decode_running_max_moves_for_some_heads_only():
         for h in (3, 40, 77, 110):
             u = q[b, 0, h, :nr]
             row[:nr] += 14.0 * u / np.linalg.norm(u)
-        raw[b, 60] = row
-    data["kv_raw"] = W.bf16_bits(raw)
+        cmp[b, idx_o[b].max()] = row
+    data["kv_cmp"] = W.bf16_bits(cmp)
     idx, out = run_decode(wl, data)
-    idx_o, out_o = oracle_decode(wl, data, [0, 1])
-    assert np.array_equal(idx.cpu().numpy(), idx_o), "top-k indices differ"
-    assert_close(host64(out), out_o, wl.dtype, "decode with an aligned window row")
+    idx_w, out_o = oracle_decode(wl, data, [0, 1])
+    assert np.array_equal(idx.cpu().numpy(), idx_w), "top-k indices differ"
+    assert_close(host64(out), out_o, wl.dtype, "decode with an aligned selected entry")
 
 
 def test_decode_extended_rope_past_the_original_context():
