@@ -27,11 +27,10 @@
 //                               O   += P(j) V(j) (N = 256, A = P from TMEM)
 //   warps 4-7: q by TMA, the row list (the window's rows first: their
 //              leading tiles are gathered while the selection's indices
-//              load), then the gather: TMA tile::gather4 (four rows x 64
-//              dims per instruction) of the CTA's half of each row into
-//              128B-swizzled chunks.  A gather4 holds its
-//              warp for ~60 ns (one warp moves ~16 GB/s), so four warps
-//              issue: warp 4 + (2 (i % 2) + c) fetches chunk c of tile i.
+//              load), then the gather: 16-byte cp.async of the CTA's half
+//              of each row into 128B-swizzled chunks (FP8 codes: TMA
+//              tile::gather4); warp 4 + (2 (i % 2) + c) fetches chunk c of
+//              tile i.
 //   warps 0-3: one head per thread (= TMEM lane): this CTA's partial logits
 //              of each tile, rounded to fp16, out to the partner (st.async
 //              into its receive buffers), the partner's in; online softmax
@@ -263,7 +262,8 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kApSlots; ++s) {
-      mbar_init(&sm.full[s], kFp8 ? 2 : 1);  // expect_tx + the chunk's bytes (FP8: 2 expanders)
+      // bf16: the 32 lanes of the gathering warp (cp.async arrivals); FP8: the 2 expanders
+      mbar_init(&sm.full[s], kFp8 ? 2 : 32);
       mbar_init(&sm.empty[s], 1);
       mbar_init(&sm.stage[s], 1);  // FP8: expect_tx + the codes' bytes
     }
@@ -328,30 +328,34 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
   // known without the selection, lead the first splits.
   auto tile_row0 = [&](int i) { return (split + i * S) * kApTile; };
 
-  // One chunk's gathers (the slot is free): bf16 rows, lane l fetches rows
-  // 4 (l & 15) .. + 3 of the tile, 64-dim half l >> 4; groups at or past
-  // n_rows are zero-filled, so that masked rows hold finite values.
+  // One chunk's gathers (the slot is free), bf16 rows: 16-byte cp.async, lane
+  // l copies unit l % 8 of rows 4k + l / 8 (k = 0..15), both 64-dim halves,
+  // into the 128B-swizzled layout (a warp instruction reads four whole
+  // 128-byte row segments); rows at or past n_rows are zero-filled, so that
+  // masked rows hold finite values.  Each lane arrives on the slot's full
+  // barrier when its copies have landed (32 arrivals).
   auto gather_chunk_bf16 = [&](int i, int ck, int n_rows, int pw) {
     const int n = 2 * i + ck;
     const int slot = n % kApSlots;
-    const int h = lane >> 4, rg = lane & 15;
-    const int g = tile_row0(i) + 4 * rg;  // list index of the group's first row
-    const bool valid = g < n_rows;
-    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-    uint8_t* dst = ring + slot * kApChunkBytes + h * (kApChunkBytes / 2) + rg * 512;
-    if (!valid) {
-#pragma unroll
-      for (int u = 0; u < 32; ++u) reinterpret_cast<uint4*>(dst)[u] = make_uint4(0u, 0u, 0u, 0u);
-      fence_proxy_async_shared();  // read by the MMA (async proxy)
+    const uint32_t cbase = smem_u32(ring + slot * kApChunkBytes);
+    const int g0 = tile_row0(i);
+    const int u = lane & 7, rsub = lane >> 3;
+    const size_t col = (size_t)(dim0 + ck * 128) * 2 + (size_t)u * 16;  // byte in the row
+    if (lane == 0) sm.last_n[slot] = n;
+#pragma unroll 4
+    for (int k = 0; k < 16; ++k) {
+      const int r = 4 * k + rsub;  // row of the chunk
+      const int g = g0 + r;
+      const bool valid = g < n_rows;
+      const char* src = reinterpret_cast<const char*>(a.q);  // read only when valid
+      if (valid)
+        src = reinterpret_cast<const char*>(g < pw ? a.kv_raw : a.kv_cmp) +
+              (size_t)sm.rows[g] * (kApDim * 2) + col;
+      const uint32_t d0 = cbase + (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4));
+      cp_async16(d0, src, valid);
+      cp_async16(d0 + kApChunkBytes / 2, src + 128, valid);
     }
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)__popc(vmask) * 512u);
-      sm.last_n[slot] = n;
-    }
-    if (valid)
-      tma_gather4(dst, g < pw ? &tm_raw : &tm_cmp, &sm.full[slot], dim0 + ck * 128 + h * 64,
-                  sm.rows[g], sm.rows[g + 1], sm.rows[g + 2], sm.rows[g + 3]);
+    cp_async_arrive(&sm.full[slot]);
   };
   // FP8: lanes 0-15 each gather the codes of rows 4l .. 4l + 3 (128 B a row)
   // into the upper half of the slot; the rows' scales go to sm.scl.
@@ -867,6 +871,7 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
       if (!okp) break;
       gather_chunk_bf16(i, ck, n_rows, pw);
     }
+    cp_async_wait_all();  // every copy into shared memory lands before the CTA may exit
   } else if (warp == 8 && lane == 0) {
     // ======================= MMA issuer
     constexpr uint32_t id_qk = idesc_bf16_f32(128, kApTile);
@@ -935,6 +940,7 @@ __global__ void __launch_bounds__(kFp8 ? kApThreadsFp8 : kApThreads, 1)
           }
         }
         if (!okm) break;
+        if (!kFp8) fence_proxy_async_shared();  // written by cp.async (generic proxy), read by the MMA
         tc_fence_after();
         const uint64_t bd0 = sw128_desc(smem_u32(ring + slot * kApChunkBytes), 16, 1024);
         const uint32_t a0 = t_q + (uint32_t)(ck * 64);  // q dims ck*128.. as bf16 pairs
