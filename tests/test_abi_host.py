@@ -136,6 +136,41 @@ def test_validation_before_device(lib):
     assert "aligned" in lib.csa_last_error_detail().decode()
 
 
+def test_validation_of_the_append_quantize_fp8_and_reuse_calls(lib):
+    """The calls beyond the layer's steps reject bad arguments on the host."""
+    p = csa.Params().c()
+    pp = ctypes.byref(p)
+    P = ctypes.c_void_p
+    # csa_compress_append: negative sizes, NULL range arrays, misaligned cache
+    assert lib.csa_compress_append(pp, 1, P(16), P(16), P(16), 0, 64, P(16), P(16), 8, P(16), 4,
+                                   None, None, 0, None) == 3           # B = 0
+    assert lib.csa_compress_append(pp, 1, P(16), P(16), P(16), 1, 64, P(16), P(16), -1, P(16), 4,
+                                   None, None, 0, None) == 3           # max_new < 0
+    assert lib.csa_compress_append(pp, 1, P(16), P(16), P(16), 1, 64, None, P(16), 8, P(16), 4,
+                                   None, None, 0, None) == 1           # t_old NULL
+    assert lib.csa_compress_append(pp, 1, P(16), P(16), P(16), 1, 64, P(16), P(16), 8, P(24), 4,
+                                   None, None, 0, None) == 2           # kv_cmp misaligned
+    assert lib.csa_compress_append(pp, 1, P(16), P(16), P(16), 1, 64, P(16), P(16), 8, P(16), 4,
+                                   P(16), None, 8, None) == 1          # kv_raw without raw_pos0
+    # csa_quantize_fp8: unsupported row width, NULL scales
+    assert lib.csa_quantize_fp8(1, P(16), 4, 48, P(16), P(16), None) == 3
+    assert lib.csa_quantize_fp8(1, P(16), 4, 512, P(16), None, None) == 1
+    assert lib.csa_quantize_fp8(1, P(16), 0, 512, None, None, None) == 0  # nothing to do
+    # FP8 attention: a shape off the tensor-core path; NULL scales
+    q = csa.Params(n_heads=64).c()
+    assert lib.csa_sparse_attn_fp8(ctypes.byref(q), P(16), P(16), P(16), P(16), P(16), 10, P(16),
+                                   P(16), P(16), P(16), 4, P(16), 1, 1, P(16), None, 0, None) == 3
+    assert lib.csa_sparse_attn_fp8(pp, P(16), P(16), P(16), None, P(16), 10, P(16), P(16), P(16),
+                                   P(16), 4, P(16), 1, 1, P(16), None, 0, None) == 1
+    assert lib.hca_attn_fp8(pp, P(16), P(16), P(16), P(16), P(16), 10, P(16), None, P(16), P(16),
+                            4, P(16), 1, 1, P(16), None, 0, None) == 1
+    # csa_reuse_attn: no layers, or layers x B x Tq beyond one grid dimension
+    assert lib.csa_reuse_attn(pp, 1, 0, P(16), P(16), P(16), P(16), 10, P(16), P(16), P(16), 4,
+                              P(16), 1, 1, P(16), None, 0, None) == 3
+    assert lib.csa_reuse_attn(pp, 1, 2, P(16), P(16), P(16), P(16), 10, P(16), P(16), P(16), 4,
+                              P(16), 40000, 1, P(16), None, 0, None) == 3
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(L, "_lib", None)
