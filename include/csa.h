@@ -54,6 +54,11 @@
  *   (and its writes to be visible) before its first access to global
  *   memory, so stream order holds for all data.  The attention calls with
  *   few query tokens launch thread-block clusters.
+ * Tracing: every call that validates, sizes or launches (all but the plain
+ *   getters and setters) is an NVTX v3 range in the domain "csa", named
+ *   after the call and open for its host-side duration, early rejections
+ *   included.  Without a tool attached (Nsight Systems, or a library named
+ *   by NVTX_INJECTION64_PATH) a range costs one branch.
  */
 #ifndef CSA_H_
 #define CSA_H_

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -27,6 +28,31 @@ namespace csa {
 namespace {
 
 thread_local char g_detail[512] = "";
+
+// Tracing: every call of the C ABI that validates, plans or launches opens an
+// NVTX range named after itself, in the domain "csa", for its host-side
+// duration.  With no tool attached an NVTX call is one test of a function
+// pointer; under Nsight Systems (or any NVTX injection library) the ranges
+// show which call launched which kernels.
+nvtxDomainHandle_t trace_domain() {
+  static const nvtxDomainHandle_t d = nvtxDomainCreateA("csa");
+  return d;
+}
+
+struct CallRange {
+  explicit CallRange(const char* name) {
+    nvtxEventAttributes_t ev;
+    std::memset(&ev, 0, sizeof(ev));
+    ev.version = NVTX_VERSION;
+    ev.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+    ev.messageType = NVTX_MESSAGE_TYPE_ASCII;
+    ev.message.ascii = name;
+    nvtxDomainRangePushEx(trace_domain(), &ev);
+  }
+  ~CallRange() { nvtxDomainRangePop(trace_domain()); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 csa_status_t fail(csa_status_t st, const char* fmt, ...) {
   va_list ap;
@@ -440,6 +466,7 @@ CSA_API uint64_t csa_launch_count(void) {
 
 CSA_API csa_status_t csa_workspace_size(const csa_params_t* p, csa_op_t op, int32_t B, int32_t Tq,
                                 int32_t n_max, size_t* bytes) {
+  const CallRange trace("csa_workspace_size");
   if (bytes == nullptr) return fail(CSA_ERR_INVALID_ARGUMENT, "bytes is NULL");
   CSA_CHECK(check_params(p));
   CSA_CHECK(check_sizes(B, Tq, n_max));
@@ -495,6 +522,7 @@ static CompressArgs compress_args(const csa_params_t* p, const void* x, const vo
 CSA_API csa_status_t csa_compress(const csa_params_t* p, csa_dtype_t dtype, const void* x,
                           const void* gate, int32_t B, int32_t T, void* kv_cmp_out,
                           void* kv_raw_rot_out, void* stream) {
+  const CallRange trace("csa_compress");
   CSA_CHECK(check_params(p));
   CSA_CHECK(check_dtype(dtype));
   CSA_CHECK(check_ptr(x, "x"));
@@ -522,6 +550,7 @@ CSA_API csa_status_t csa_compress_append(const csa_params_t* p, csa_dtype_t dtyp
                                          int32_t max_new, void* kv_cmp, int32_t n_cap,
                                          void* kv_raw, const int32_t* raw_pos0, int32_t raw_cap,
                                          void* stream) {
+  const CallRange trace("csa_compress_append");
   CSA_CHECK(check_params(p));
   CSA_CHECK(check_dtype(dtype));
   if (B < 1 || B > 65535 || L < 0 || max_new < 0 || n_cap < 0 || raw_cap < 0)
@@ -684,6 +713,7 @@ CSA_API csa_status_t csa_index_scores(const csa_params_t* p, csa_dtype_t dtype, 
                               const float* w, const void* k_idx, const int32_t* q_pos,
                               const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
                               float* scores, void* stream) {
+  const CallRange trace("csa_index_scores");
   CSA_CHECK(check_params(p));
   CSA_CHECK(check_dtype(dtype));
   CSA_CHECK(check_indexer_shape(p));
@@ -702,6 +732,7 @@ CSA_API csa_status_t csa_index_scores(const csa_params_t* p, csa_dtype_t dtype, 
 CSA_API csa_status_t csa_topk_select(const csa_params_t* p, const float* scores, const int32_t* q_pos,
                              const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
                              int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange trace("csa_topk_select");
   CSA_CHECK(check_params(p));
   CSA_CHECK(check_topk(p));
   CSA_CHECK(check_sizes(B, Tq, n_max));
@@ -719,6 +750,7 @@ CSA_API csa_status_t csa_index_topk(const csa_params_t* p, csa_dtype_t dtype, co
                             const float* w, const void* k_idx, const int32_t* q_pos,
                             const int32_t* n_cmp, int32_t B, int32_t Tq, int32_t n_max,
                             int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange trace("csa_index_topk");
   CSA_CHECK(check_params(p));
   CSA_CHECK(check_dtype(dtype));
   CSA_CHECK(check_indexer_shape(p));
@@ -893,6 +925,7 @@ CSA_API csa_status_t csa_sparse_attn(const csa_params_t* p, csa_dtype_t dtype, c
                              const int32_t* n_raw, int32_t raw_max, const float* sink,
                              int32_t B, int32_t Tq, void* out, void* ws, size_t ws_bytes,
                              void* stream) {
+  const CallRange trace("csa_sparse_attn");
   CSA_CHECK(attn_common_checks(p, dtype, q, q_pos, kv_cmp, n_max, kv_raw, raw_pos0, n_raw,
                                raw_max, sink, B, Tq, out));
   CSA_CHECK(check_topk(p));
@@ -911,6 +944,7 @@ CSA_API csa_status_t csa_reuse_attn(const csa_params_t* p, csa_dtype_t dtype, in
                                     const int32_t* raw_pos0, const int32_t* n_raw,
                                     int32_t raw_max, const float* sink, int32_t B, int32_t Tq,
                                     void* out, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange trace("csa_reuse_attn");
   CSA_CHECK(attn_common_checks(p, dtype, q, q_pos, kv_cmp, n_max, kv_raw, raw_pos0, n_raw,
                                raw_max, sink, B, Tq, out));
   CSA_CHECK(check_topk(p));
@@ -944,6 +978,7 @@ CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const vo
                       int32_t n_max, const void* kv_raw, const int32_t* raw_pos0,
                       const int32_t* n_raw, int32_t raw_max, const float* sink, int32_t B,
                       int32_t Tq, void* out, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange trace("hca_attn");
   CSA_CHECK(attn_common_checks(p, dtype, q, q_pos, kv_cmp, n_max, kv_raw, raw_pos0, n_raw,
                                raw_max, sink, B, Tq, out));
   CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
@@ -961,6 +996,7 @@ CSA_API csa_status_t hca_attn(const csa_params_t* p, csa_dtype_t dtype, const vo
 // ---------------------------------------------------------------------------
 CSA_API csa_status_t csa_quantize_fp8(csa_dtype_t dtype, const void* rows, int64_t n, int32_t d,
                                       uint8_t* codes, float* scales, void* stream) {
+  const CallRange trace("csa_quantize_fp8");
   CSA_CHECK(check_dtype(dtype));
   if (n < 0 || d < 8 || d > 1024 || (d & 31))
     return fail(CSA_ERR_UNSUPPORTED_SHAPE, "n=%lld d=%d: d a multiple of 32 in [32, 1024]",
@@ -1007,6 +1043,7 @@ CSA_API csa_status_t csa_sparse_attn_fp8(const csa_params_t* p, const void* q,
                                          const int32_t* n_raw, int32_t raw_max, const float* sink,
                                          int32_t B, int32_t Tq, void* out, void* ws,
                                          size_t ws_bytes, void* stream) {
+  const CallRange trace("csa_sparse_attn_fp8");
   CSA_CHECK(attn_fp8_checks(p, false, q, q_pos, kv_cmp, cmp_scale, n_max, kv_raw, raw_scale,
                             raw_pos0, n_raw, raw_max, sink, B, Tq, out));
   CSA_CHECK(check_topk(p));
@@ -1026,6 +1063,7 @@ CSA_API csa_status_t hca_attn_fp8(const csa_params_t* p, const void* q, const in
                                   const int32_t* n_raw, int32_t raw_max, const float* sink,
                                   int32_t B, int32_t Tq, void* out, void* ws, size_t ws_bytes,
                                   void* stream) {
+  const CallRange trace("hca_attn_fp8");
   CSA_CHECK(attn_fp8_checks(p, true, q, q_pos, kv_cmp, cmp_scale, n_max, kv_raw, raw_scale,
                             raw_pos0, n_raw, raw_max, sink, B, Tq, out));
   CSA_CHECK(check_ptr(n_cmp, "n_cmp"));
@@ -1110,6 +1148,7 @@ CSA_API csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t d
                                             const int32_t* q_pos, const int32_t* n_cmp,
                                             int32_t B, int32_t Tq, int32_t n_max,
                                             int32_t* idx_out, void* stream) {
+  const CallRange trace("csa_index_topk_noalloc");
   CSA_CHECK(check_params(p));
   CSA_CHECK(check_dtype(dtype));
   CSA_CHECK(check_indexer_shape(p));
@@ -1141,6 +1180,7 @@ CSA_API csa_status_t csa_index_topk_noalloc(const csa_params_t* p, csa_dtype_t d
 static std::atomic<int32_t> g_last_site{0};
 
 CSA_API csa_status_t csa_poll_device_error(void* stream) {
+  const CallRange trace("csa_poll_device_error");
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
   int v = 0, site = 0;
