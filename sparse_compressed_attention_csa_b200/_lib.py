@@ -64,11 +64,17 @@ class Params:
     rope_beta_slow: float = 1.0   # YaRN alpha
 
     def c(self) -> csa_params_t:
-        sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
-        return csa_params_t(self.d, self.rope_dim, self.theta, sc, self.n_heads, self.idx_heads,
-                            self.idx_dim, self.topk, self.window, self.width, self.stride,
-                            self.pos_offset, self.rope_factor, self.rope_orig_ctx,
-                            self.rope_beta_fast, self.rope_beta_slow)
+        """The C struct, built once per (immutable) parameter set; the
+        library only reads it during a call."""
+        cs = self.__dict__.get("_c")
+        if cs is None:
+            sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+            cs = csa_params_t(self.d, self.rope_dim, self.theta, sc, self.n_heads,
+                              self.idx_heads, self.idx_dim, self.topk, self.window, self.width,
+                              self.stride, self.pos_offset, self.rope_factor, self.rope_orig_ctx,
+                              self.rope_beta_fast, self.rope_beta_slow)
+            object.__setattr__(self, "_c", cs)
+        return cs
 
 
 _lib = None
@@ -136,14 +142,21 @@ def _check(st: int):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # a plain int: the c_void_p argtypes convert it
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream):
+    """The cudaStream_t of `stream`, or of the current stream of the current
+    device (read through torch's raw-stream query, which skips building a
+    Stream object on every call)."""
     import torch
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    if stream is not None:
+        return stream.cuda_stream
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return raw(torch._C._cuda_getDevice())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _dtype_code(t):
@@ -170,10 +183,21 @@ def _req(t, name, dtype=None, ndim=None):
     return t
 
 
+_ws_sizes = {}
+
+
 def csa_workspace_size(p: Params, op: int, B: int, Tq: int, n_max: int) -> int:
-    n = ctypes.c_size_t(0)
-    _check(_load().csa_workspace_size(ctypes.byref(p.c()), op, B, Tq, n_max, ctypes.byref(n)))
-    return int(n.value)
+    """Bytes of workspace the call `op` needs (a pure function of the
+    arguments and the current device, so answers are kept per device)."""
+    import torch
+    key = (p, op, B, Tq, n_max, torch.cuda.current_device() if torch.cuda.is_available() else -1)
+    nb = _ws_sizes.get(key)
+    if nb is None:
+        n = ctypes.c_size_t(0)
+        _check(_load().csa_workspace_size(ctypes.byref(p.c()), op, B, Tq, n_max,
+                                          ctypes.byref(n)))
+        nb = _ws_sizes[key] = int(n.value)
+    return nb
 
 
 def csa_compress(p: Params, x, gate, kv_cmp_out, kv_raw_rot_out=None, stream=None):

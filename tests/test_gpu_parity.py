@@ -133,9 +133,14 @@ def test_hca_decode_128k_bs16():
 
 
 def test_csa_prefill_8k():
+    # the first rows (nothing or few entries visible), a block boundary, the
+    # last rows, and 256 rows drawn uniformly: every query token runs its own
+    # CTA pairs, so the sample covers 256 independent launches' worth of
+    # work at full size
     rng = np.random.default_rng(1234)
     rows = np.unique(np.concatenate([np.arange(0, 16), np.arange(4095, 4104),
-                                     np.arange(8176, 8192), rng.integers(0, 8192, 64)]))
+                                     np.arange(8176, 8192), rng.integers(0, 8192, 256)]))
+    assert rows.size >= 256
     check_prefill(W.CSA_PREFILL_8K, rows)
 
 
@@ -365,13 +370,32 @@ def test_topk_select_adversarial_scores(n, k, rows, visible):
         assert np.array_equal(got[b, 0], want), b
 
 
-def test_deterministic_repeat():
-    wl = W.CSA_DECODE_64K.replace(B=2, T=9000, seed=30)
+def _bits(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t
+
+
+@pytest.mark.parametrize("case", ["decode_64k", "decode_long_rows", "hca_decode", "prefill"])
+def test_deterministic_repeat(case):
+    # ten runs on the same inputs give bitwise-identical outputs and the same
+    # top-k: the pair's partial-logit exchange, the cluster top-k's exchanges
+    # and the split-KV merge all combine in a fixed order
+    wl, run = {
+        "decode_64k": (W.CSA_DECODE_64K.replace(B=2, T=9000, seed=30), run_decode),
+        # rows of 100,000 entries: the wide top-k cluster and many KV splits
+        "decode_long_rows": (W.CSA_DECODE_1M.replace(B=2, T=4 * 100000 + 4, seed=32), run_decode),
+        "hca_decode": (W.HCA_DECODE_128K.replace(B=3, T=128 * 700 + 5, seed=33), run_hca),
+        "prefill": (W.CSA_PREFILL_8K.replace(T=1203, topk=256, seed=34), run_prefill),
+    }[case]
     data = W.generate(wl)
-    i1, o1 = run_decode(wl, data)
-    i2, o2 = run_decode(wl, data)
-    assert torch.equal(i1, i2)
-    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+    def once():
+        r = run(wl, data)
+        return [_bits(x) for x in (r if isinstance(r, tuple) else (r,))]
+
+    first = once()
+    for _ in range(9):
+        for a, b in zip(first, once()):
+            assert torch.equal(a, b), case
 
 
 def test_device_bounds_error_is_reported():
