@@ -190,9 +190,11 @@ def algorithmic_work(wl):
                         "flops": int(4 * n_q * H * n_rows * d)}
     if wl.reuse_layers:
         g["reuse_attn"] = {k: wl.reuse_layers * v for k, v in g["sparse_attn"].items()}
-    # the step's own bytes: scores and indices stay between its kernels (each
-    # Reuse layer reads the selection again)
-    g["step"] = {"bytes": sum(v["bytes"] for v in g.values()) - 2 * scores - 2 * sel}
+    # the step's own bytes: the scores stay between its kernels; the
+    # selection is an output of the step (the caller's index buffer), counted
+    # once, not again for the attention's read of it (each Reuse layer's read
+    # is counted)
+    g["step"] = {"bytes": sum(v["bytes"] for v in g.values()) - 2 * scores - sel}
     return g
 
 
