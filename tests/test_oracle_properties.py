@@ -122,3 +122,43 @@ def test_fp8_rows_decode_within_half_a_code_step(n, d, log_mag, zero_row, seed):
             assert np.abs(back[r]).max() == 448.0 * float(scales[r])
         else:
             assert scales[r] == 1.0 and np.all(back[r] == 0.0)
+
+
+@SETTINGS
+@given(H=st.integers(1, 4), dI=st.integers(1, 8), N=st.integers(0, 20),
+       seed=st.integers(0, 2 ** 31))
+def test_index_scores_integer_inputs_exact(H, dI, N, seed):
+    # integer keys and queries with power-of-two weights: every score is an
+    # exact binary value, so the oracle and the brute force agree bit for bit
+    rng = np.random.default_rng(seed)
+    q = rng.integers(-8, 9, (H, dI)).astype(np.float64)
+    w = 2.0 ** rng.integers(-2, 3, H)
+    k = rng.integers(-8, 9, (N, dI)).astype(np.float64)
+    got = oracle.index_scores(q[None], w[None], k)[0]
+    assert got.tolist() == brute.scores(q.tolist(), w.tolist(), k.tolist())
+
+
+_YARN = st.builds(oracle.YaRN, theta=st.sampled_from([10000.0, 160000.0, 500.0]),
+                  factor=st.sampled_from([1.0, 4.0, 16.0]),
+                  orig_ctx=st.sampled_from([40, 4096, 65536]))
+
+
+@SETTINGS
+@given(spec=_YARN, rope_dim=st.sampled_from([4, 16, 64]))
+def test_yarn_frequencies_lie_between_the_scaled_and_the_original(spec, rope_dim):
+    # each pair's frequency is a blend of f / s and f with a weight in
+    # [0, 1]: it lies between the two, and it falls with the pair index
+    f = oracle.rope_freqs(rope_dim, spec.theta)
+    fy = oracle.rope_freqs(rope_dim, spec)
+    assert np.all(fy <= f * (1 + 1e-15)) and np.all(fy >= f / spec.factor * (1 - 1e-15))
+    assert np.all(np.diff(fy) < 0)
+
+
+@SETTINGS
+@given(spec=_YARN, a=st.integers(-200000, 200000), b=st.integers(-200000, 200000),
+       seed=st.integers(0, 2 ** 31))
+def test_yarn_rotations_compose(spec, a, b, seed):
+    x = np.random.default_rng(seed).standard_normal(8 + 2)
+    ab = oracle.rope(oracle.rope(x, a, 8, spec), b, 8, spec)
+    np.testing.assert_allclose(ab, oracle.rope(x, a + b, 8, spec), rtol=0, atol=1e-9)
+    assert np.array_equal(ab[:2], x[:2])
