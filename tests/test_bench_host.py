@@ -53,3 +53,38 @@ def test_prefill_flops():
     assert g["sparse_attn"]["flops"] == 4 * 128 * rows * 512
     assert g["index_scores"]["flops"] == 2 * sum(vis) * 64 * 128
     assert round((g["sparse_attn"]["flops"] + g["index_scores"]["flops"]) / 1e12, 3) == 2.058
+
+
+def _run_bench(args, env_extra=None, timeout=300):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **(env_extra or {}))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], cwd=root, env=env,
+                       capture_output=True, text=True, timeout=timeout)
+    assert r.returncode == 0, r.stdout + r.stderr
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    return lines
+
+
+def test_reference_arm_prints_one_complete_line():
+    # the oracle timed on the host cores on the headline's config: one JSON
+    # line with the same metric, unit and direction as the CUDA arm, its own
+    # cpu_baseline, and an e2e entry that moves no bytes
+    (line,) = _run_bench(["--impl", "reference", "--steps", "2", "--warmup", "3"])
+    assert line["impl"] == "reference"
+    assert line["unit"] == "query-heads/s" and line["higher_is_better"] is True
+    assert line["metric"].startswith("CSA decode query-heads/s")
+    assert line["config"]["workload"] == "csa_decode_bs32_ctx65536"
+    assert line["value"] > 0 and line["dtype"] == "f64" and line["warmup"] >= 3
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "query-heads/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    assert _run_bench(["--impl", "reference", "--steps", "2", "--warmup", "3"],
+                      {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
