@@ -162,3 +162,33 @@ def test_yarn_rotations_compose(spec, a, b, seed):
     ab = oracle.rope(oracle.rope(x, a, 8, spec), b, 8, spec)
     np.testing.assert_allclose(ab, oracle.rope(x, a + b, 8, spec), rtol=0, atol=1e-9)
     assert np.array_equal(ab[:2], x[:2])
+
+
+@SETTINGS
+@given(ws=st.sampled_from([(8, 4), (2, 2), (5, 3), (16, 16), (4, 1)]), T=st.integers(0, 120),
+       cuts=st.lists(st.integers(0, 120), max_size=12), back=st.integers(0, 5),
+       seed=st.integers(0, 2 ** 31))
+def test_append_at_any_cuts_equals_whole_sequence(ws, T, cuts, back, seed):
+    # tokens arrive in bursts cut anywhere (empty bursts too), each burst
+    # handed a window that starts at most `back` tokens before what it needs:
+    # the appended entries and raw rows, in order, are the whole sequence's
+    width, stride = ws
+    rng = np.random.default_rng(seed)
+    d, r = 4, 2
+    x, g = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    bounds = sorted({0, T, *[c for c in cuts if c <= T]})
+    ents, raws, seen = [], [], 0
+    for t_old, t_new in zip(bounds[:-1], bounds[1:]):
+        j_first = oracle.n_compressed(t_old, width, stride)
+        lo = max(0, min(stride * j_first, t_old) - back)
+        j0, e, raw = oracle.compress_append(x[lo:t_new], g[lo:t_new], lo, t_old, t_new, width,
+                                            stride, r, THETA)
+        assert j0 == seen
+        seen += e.shape[0]
+        ents.append(e)
+        raws.append(raw)
+    full = oracle.compress(x, g, width, stride, r, THETA)
+    assert seen == full.shape[0]
+    np.testing.assert_array_equal(np.concatenate(ents) if ents else np.zeros((0, d)), full)
+    np.testing.assert_array_equal(np.concatenate(raws) if raws else np.zeros((0, d)),
+                                  oracle.rotate_raw(x, 0, r, THETA))
