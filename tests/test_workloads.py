@@ -64,3 +64,19 @@ def test_positions_and_window_bookkeeping():
     p = W.generate(SMALL_PREFILL)
     assert np.array_equal(p["q_pos"][0], np.arange(SMALL_PREFILL.T))
     assert "kv_cmp" not in p  # prefill pools its own entries on the path
+
+
+def test_indexer_inputs_keep_every_fp32_sum_exact():
+    # worst case over the recipe: a dot product of d_I integers of magnitude
+    # <= r is at most d_I r^2; the score adds H_I of them times a weight of
+    # at most 2^e_max; every value is a multiple of 2^e_min.  Below 2^24
+    # units of 2^e_min, every partial sum in fp32 is exact, so the GPU's
+    # scores (and the top-k decided on them) must equal the oracle's bit
+    # for bit, whatever order the sums take
+    for wl in (W.CSA_DECODE_64K, W.CSA_DECODE_1M, W.CSA_PREFILL_8K, W.TINY_F32, W.CSA2_DECODE):
+        r = wl.int_range
+        e_min, e_max = min(wl.w_exps), max(wl.w_exps)
+        dot = wl.idx_dim * r * r
+        assert dot < 2 ** 24, wl.name                       # the MMA's fp32 accumulation
+        score_units = wl.idx_heads * dot * 2 ** (e_max - e_min)
+        assert score_units < 2 ** 24, wl.name               # the weighted head sum
